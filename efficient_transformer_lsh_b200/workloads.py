@@ -1,0 +1,141 @@
+"""Seeded synthetic workloads for LSH self-attention.
+
+This module only draws random numbers and rounds them to the input dtype.
+It holds none of the attention arithmetic, so the CUDA path and the CPU
+oracle can both take their inputs from it without sharing any of the method.
+
+Recipe (one per named workload):
+  * generator: numpy PCG64 seeded with ``20200 + index``; ``SeedSequence.spawn``
+    gives independent streams for qk, v, R and dO;
+  * values are drawn in float64 and rounded once to the input dtype
+    (round-to-nearest-even); bf16 values are returned as float32 arrays whose
+    values are exactly representable in bf16, so widening them is exact;
+  * qk, v, dO have shape [B, H, L, d]; R has shape [n_rounds, d, n_buckets/2]
+    (one random rotation per hash round, shared by every batch and head);
+  * ``qk="mixture"`` draws 256 cluster centres ~ N(0, I) and gives every token
+    a uniformly chosen centre plus N(0, 0.1^2) noise, which makes bucket
+    occupancy uneven the way real text does; every other array is N(0, 1).
+
+The sizes mirror the experiments named on the Reformer pages (64K-token
+enwik8, 12K-token imagenet-64, half-million-token sequences); the datasets
+themselves are not used: these synthetic arrays stand in for them.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, Optional
+
+import numpy as np
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    index: int
+    dtype: str          # "f32" or "bf16"
+    B: int
+    H: int
+    L: int
+    d: int
+    n_buckets: int
+    chunk: int
+    n_rounds: int
+    causal: bool
+    backward: bool
+    qk: str = "normal"  # "normal" or "mixture"
+    n_clusters: int = 256
+    cluster_sigma: float = 0.1
+
+    @property
+    def tokens(self) -> int:
+        """Tokens per call, B*L (the unit of the tokens/s metric)."""
+        return self.B * self.L
+
+    @property
+    def rows(self) -> int:
+        """Token-heads, B*H*L."""
+        return self.B * self.H * self.L
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.d))
+
+    def with_sizes(self, **kw) -> "Workload":
+        """Same recipe at other sizes (parity cases the oracle finishes in seconds)."""
+        return dataclasses.replace(self, **kw)
+
+    def describe(self) -> Dict[str, object]:
+        return {
+            "workload": self.name, "dtype": self.dtype, "B": self.B, "H": self.H,
+            "L": self.L, "d_head": self.d, "n_buckets": self.n_buckets,
+            "chunk": self.chunk, "n_rounds": self.n_rounds, "causal": self.causal,
+            "pass": "fwd+bwd" if self.backward else "fwd", "qk": self.qk,
+        }
+
+
+WORKLOADS: Dict[str, Workload] = {
+    w.name: w for w in [
+        Workload("toy-f32-L1024", 1, "f32", 1, 1, 1024, 64, 32, 64, 1, False, False),
+        Workload("toy-f32-L1024-fullchunk", 1, "f32", 1, 1, 1024, 64, 32, 1024, 1, False, False),
+        Workload("batch-bf16-8x8x4096", 2, "bf16", 8, 8, 4096, 64, 64, 64, 2, True, False),
+        Workload("enwik8-64k-bf16", 3, "bf16", 1, 8, 65536, 64, 1024, 64, 4, True, True,
+                 qk="mixture"),
+        Workload("imagenet64-12k-bf16", 4, "bf16", 4, 8, 12288, 64, 192, 64, 8, True, True),
+        Workload("halfmillion-bf16", 5, "bf16", 1, 2, 524288, 64, 8192, 64, 1, True, False),
+    ]
+}
+
+# The throughput workload: 64K tokens, 8 heads, 4 hash rounds, forward + backward.
+HEADLINE = "enwik8-64k-bf16"
+
+
+def round_to_bf16(a: np.ndarray) -> np.ndarray:
+    """Round float64/float32 values to the nearest bf16 (ties to even).
+
+    Returns float32 holding exactly representable bf16 values.
+    """
+    f = np.ascontiguousarray(a, dtype=np.float32)
+    bits = f.view(np.uint32).astype(np.uint64)
+    bits = (bits + 0x7FFF + ((bits >> 16) & 1)) & 0xFFFF0000
+    return bits.astype(np.uint32).view(np.float32)
+
+
+def _to_dtype(a: np.ndarray, dtype: str) -> np.ndarray:
+    if dtype == "f32":
+        return a.astype(np.float32)
+    if dtype == "bf16":
+        return round_to_bf16(a)
+    raise ValueError(dtype)
+
+
+def generate(w: Workload, seed: Optional[int] = None, with_grad: Optional[bool] = None):
+    """Draw the inputs of workload ``w``.
+
+    Returns a dict of float32 numpy arrays: qk, v, R and (when a backward pass
+    is wanted) dO. Values are exactly representable in ``w.dtype``.
+    """
+    if seed is None:
+        seed = 20200 + w.index
+    if with_grad is None:
+        with_grad = w.backward
+    s_qk, s_v, s_r, s_do = np.random.SeedSequence(seed).spawn(4)
+    shape = (w.B, w.H, w.L, w.d)
+    g = np.random.Generator(np.random.PCG64(s_qk))
+    if w.qk == "mixture":
+        centres = g.standard_normal((w.n_clusters, w.d))
+        assign = g.integers(0, w.n_clusters, size=shape[:-1])
+        qk = centres[assign] + w.cluster_sigma * g.standard_normal(shape)
+    elif w.qk == "normal":
+        qk = g.standard_normal(shape)
+    else:
+        raise ValueError(w.qk)
+    out = {"qk": _to_dtype(qk, w.dtype)}
+    del qk
+    out["v"] = _to_dtype(np.random.Generator(np.random.PCG64(s_v)).standard_normal(shape), w.dtype)
+    out["R"] = _to_dtype(
+        np.random.Generator(np.random.PCG64(s_r)).standard_normal(
+            (w.n_rounds, w.d, w.n_buckets // 2)), w.dtype)
+    if with_grad:
+        out["dO"] = _to_dtype(
+            np.random.Generator(np.random.PCG64(s_do)).standard_normal(shape), w.dtype)
+    return out
