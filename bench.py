@@ -1,0 +1,393 @@
+"""Throughput benchmark of Reformer LSH self-attention on B200.
+
+One step = the whole hot path over one batch of synthetic input already in
+HBM: lsh_hash -> lsh_sort -> lsh_attn_fwd (chunk attention + round combine)
+-> lsh_attn_bwd, all through the C ABI on one stream. Metric: tokens/s
+(B*L per step, summed over ranks). Prints one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the float64 CPU oracle, timed on host cores
+For N > 1 launch with torchrun; each rank runs its own independent problem
+(weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from efficient_transformer_lsh_b200.workloads import HEADLINE, WORKLOADS, generate  # noqa: E402
+
+METRIC = "LSH-attn fwd+bwd tokens/s at L=64K, 8 heads, 4 rounds; % of roofline"
+UNIT = "tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------
+# Algorithmic bytes and FLOPs (stage by stage; their sum over a step is the
+# compulsory traffic of the whole path: each stage reads its inputs once and
+# writes its outputs once).
+# ----------------------------------------------------------------------------
+
+def stage_models(w):
+    N = w.B * w.H * w.L
+    d, nr, m = w.d, w.n_rounds, w.chunk
+    e = 4 if w.dtype == "f32" else 2
+    de = d * e
+    hash_b = N * (de + 4 * nr)
+    sort_b = N * 12 * nr
+    if nr >= 2:
+        fwd_b = N * (de * (1 + 4 * nr) + 12 * nr + 4)
+    else:
+        fwd_b = N * (3 * de + 8)
+    bwd_b = N * (2 * de + 4 + nr * (3 * de + 12) + 8 * d)
+    attn_fwd_flops = w.B * w.H * nr * 4 * m * m * d * (2 * w.L / m - 1)
+    return {
+        "hash": {"bytes": hash_b, "flops": N * nr * d * w.n_buckets},
+        "sort": {"bytes": sort_b, "flops": 0},
+        "fwd": {"bytes": fwd_b, "flops": attn_fwd_flops},
+        "bwd": {"bytes": bwd_b if w.backward else 0,
+                "flops": 2.5 * attn_fwd_flops if w.backward else 0},
+    }
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+# ----------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.rows = []
+        self.proc = None
+        self.gpu_index = gpu_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        threading.Thread(target=self._read, daemon=True).start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 8:
+                self.rows.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        win = [p for t, p in self.rows if t0 - 0.15 <= t <= t1 + 0.15]
+        note = "in timed window"
+        if not win:
+            near = sorted(self.rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))[:3]
+            win = [p for _, p in near]
+            note = "nearest samples (timed window shorter than the sampling period)"
+        sm = [float(p[1]) for p in win if p[1].replace(".", "").isdigit()]
+        mx = [float(p[2]) for p in win if p[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in win for i in range(4) if p[4 + i] == "Active"})
+        pw = [float(p[3]) for p in win if p[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "power_w_max": max(pw) if pw else None, "samples": len(win), "note": note}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and the reference arm)
+# ----------------------------------------------------------------------------
+
+def oracle_sample_step(w, inp64, heads):
+    """hash + sort + forward (+ backward) of the oracle on `heads` (b=0) slices at full L."""
+    from oracle import lsh_oracle as orc
+    qk = inp64["qk"][:1, :heads]
+    v = inp64["v"][:1, :heads]
+    bucket, _ = orc.hash_buckets(qk, inp64["R"])
+    perm = orc.sort_positions(bucket)
+    O, LSE = orc.forward(qk, v, perm, w.chunk, w.causal, w.scale)
+    if w.backward:
+        orc.backward(qk, v, perm, w.chunk, w.causal, w.scale, O, LSE, inp64["dO"][:1, :heads])
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        n = 1
+    return int(n)
+
+
+def oracle_inputs(w):
+    import numpy as np
+    inp = generate(w.with_sizes(B=1))
+    return {k: a.astype(np.float64) for k, a in inp.items()}
+
+
+def cpu_baseline(w, heads):
+    inp64 = oracle_inputs(w)
+    t = time.perf_counter()
+    oracle_sample_step(w, inp64, heads)
+    dt = time.perf_counter() - t
+    frac = heads / (w.B * w.H)
+    return {"value": w.tokens * frac / dt, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "seconds": dt,
+            "sample": f"{heads} of {w.B * w.H} (batch, head) slices at full L={w.L}, all "
+                      f"{w.n_rounds} rounds, hash+sort+fwd{'+bwd' if w.backward else ''}; "
+                      f"tokens/s scaled by the slice fraction {frac:.4f}"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", 0))
+    if rank != 0:
+        return 0
+    inp64 = oracle_inputs(w)
+    heads = 1
+    for _ in range(args.warmup):
+        oracle_sample_step(w, inp64, heads)
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        oracle_sample_step(w, inp64, heads)
+        times.append(time.perf_counter() - t)
+    frac = heads / (w.B * w.H)
+    per_step = sum(times) / len(times)
+    value = w.tokens * frac / per_step
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3 / frac,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                         "sample": f"each step: {heads} of {w.B * w.H} (batch, head) slices at full "
+                                   f"L={w.L}; tokens/s scaled by {frac:.4f}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w):
+    c = w.describe()
+    c["l2"] = "no flush: each step streams >1 GB (inputs, partials, gradients), 10x the 126 MB L2"
+    return c
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS))
+    ap.add_argument("--cpu-heads", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    args.warmup = max(3, args.warmup)
+
+    import numpy as np
+    import torch
+
+    from efficient_transformer_lsh_b200 import _lib, dist
+    from efficient_transformer_lsh_b200.attention import LSHAttention
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    rank, local, world = dist.init("nccl")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    _lib.lib()
+
+    seed = dist.rank_seed(20200 + w.index, rank)
+    inp = generate(w, seed=seed)
+    td = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    host = {k: torch.from_numpy(a).to(td).pin_memory() for k, a in inp.items()}
+    d_in = {k: t.to(dev, non_blocking=True) for k, t in host.items()}
+    run = LSHAttention(w.B, w.H, w.L, w.n_buckets, w.n_rounds, w.chunk, w.causal, w.dtype, w.d,
+                       w.scale, dev)
+    stream = torch.cuda.current_stream(dev)
+    names = ["hash", "sort", "fwd", "bwd"] if w.backward else ["hash", "sort", "fwd"]
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        run.hash(d_in["qk"], d_in["R"], stream)
+        if evs is not None:
+            evs[1].record(stream)
+        run.sort(None, stream)
+        if evs is not None:
+            evs[2].record(stream)
+        run.attend(d_in["qk"], d_in["v"], None, stream)
+        if evs is not None:
+            evs[3].record(stream)
+        if w.backward:
+            run.backward(d_in["qk"], d_in["v"], d_in["dO"], None, stream)
+            if evs is not None:
+                evs[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert _lib.lsh_device_status(stream) == 0
+
+    # timed region: K whole steps, device time, max over ranks
+    gpu_index = os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local if world > 1 else 0]
+    sampler = ClockSampler(gpu_index.strip() or local)
+    sampler.start()
+    time.sleep(0.3)
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(K)]
+    launches0 = _lib.lsh_launch_count()
+    dist.barrier(dev)
+    torch.cuda.synchronize(dev)
+    t_host0 = time.time()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(K):
+        step(evs[k])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t_host1 = time.time()
+    dist.barrier(dev)
+    launches = _lib.lsh_launch_count() - launches0
+    time.sleep(0.2)
+    sampler.stop()
+    assert _lib.lsh_device_status(stream) == 0
+    t_ms = start.elapsed_time(end)
+    t_ms_max = dist.max_over_ranks(t_ms, dev)
+    ms_per_step = t_ms_max / K
+    value = world * w.tokens * K / (t_ms_max / 1e3)
+
+    stage_ms = {n: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(K))
+                for i, n in enumerate(names)}
+    models = stage_models(w)
+    peaks = load_peaks()
+    stages = {}
+    for n in names:
+        t = stage_ms[n] / 1e3
+        b, f = models[n]["bytes"], models[n]["flops"]
+        t_b = b / (peaks["hbm_gbs"] * 1e9)
+        t_f = f / (peaks["bf16_tflops"] * 1e12)
+        bound = "hbm" if t_b >= t_f else "tensor"
+        if w.dtype == "f32" and bound == "tensor":
+            bound = "alu"
+        stages[n] = {"ms": stage_ms[n], "bytes": b, "flops": f, "bound": bound,
+                     "gbs": b / t / 1e9, "tflops": f / t / 1e12,
+                     "frac": max(t_b, t_f) / t}
+    dom = max(names, key=lambda n: stage_ms[n])
+    ds = stages[dom]
+    traffic = None
+    tr_file = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tr_file):
+        try:
+            with open(tr_file) as f:
+                tr = json.load(f).get(w.name, {}).get(dom)
+            if tr is not None:
+                traffic = tr
+        except Exception:
+            traffic = None
+    if ds["bound"] == "hbm":
+        roof = {"bound": "hbm", "achieved": ds["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        roof = {"bound": ds["bound"], "achieved": ds["tflops"], "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic
+    roof["kernel"] = f"lsh_{'attn_' if dom in ('fwd', 'bwd') else ''}{dom} stage"
+    roof["peak_source"] = peaks["source"]
+    t_b = sum(models[n]["bytes"] for n in names) / (peaks["hbm_gbs"] * 1e9)
+    t_f = sum(models[n]["flops"] for n in names if n != "hash") / (peaks["bf16_tflops"] * 1e12)
+    t_star = max(t_b, t_f)
+    step_roof = {"t_star_us": t_star * 1e6, "t_step_us": ms_per_step * 1e3,
+                 "frac": t_star / (ms_per_step / 1e3),
+                 "definition": "max(algorithmic bytes / HBM peak, chunk-attention FLOPs / bf16 "
+                               "peak) over the whole step, divided by the measured step time"}
+
+    # end to end through the public API with host buffers
+    E = max(1, args.e2e_steps)
+    out_h = {"out": torch.empty(run.out.shape, dtype=run.out.dtype).pin_memory(),
+             "lse": torch.empty(run.lse.shape, dtype=torch.float32).pin_memory()}
+    if w.backward:
+        out_h["dqk"] = torch.empty(run.dqk.shape, dtype=torch.float32).pin_memory()
+        out_h["dv"] = torch.empty(run.dv.shape, dtype=torch.float32).pin_memory()
+    dev_out = {"out": run.out, "lse": run.lse, "dqk": run.dqk, "dv": run.dv}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in out_h.values())
+    dist.barrier(dev)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        for k in host:
+            d_in[k].copy_(host[k], non_blocking=True)
+        step()
+        for k in out_h:
+            out_h[k].copy_(dev_out[k], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = dist.max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e = {"value": world * w.tokens * E / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": E}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": config_of(w), "roofline": roof, "step_roofline": step_roof, "stages": stages,
+        "e2e": e2e, "gpu_launches": launches, "clocks": sampler.summary(t_host0, t_host1),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, min(args.cpu_heads, w.B * w.H))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.finish()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

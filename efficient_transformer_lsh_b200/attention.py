@@ -1,0 +1,106 @@
+"""Torch-facing driver of the C ABI: owns output and workspace buffers.
+
+PyTorch only allocates device memory and provides streams here; every step
+(hash, sort, chunk attention, round combine, backward) runs in liblsh.so.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+_TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+class LSHAttention:
+    """Reformer LSH self-attention for one fixed problem shape.
+
+    Buffers: bucket/perm [B,H,n_rounds,L] int32, out [B,H,L,d] (input dtype),
+    lse [B,H,L] float32, dqk/dv [B,H,L,d] float32, and the three workspaces.
+    """
+
+    def __init__(self, B, H, L, n_buckets, n_rounds, chunk, causal, dtype="bf16", d=64,
+                 scale: Optional[float] = None, device="cuda"):
+        self.dtype = dtype
+        self.tdtype = _TORCH_DTYPE[dtype]
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        self.p = _lib.make_problem(B, H, L, d, n_buckets, n_rounds, chunk, causal, scale, dtype)
+        self.shape = (B, H, L, d)
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.bucket = torch.empty((B, H, n_rounds, L), **i32)
+        self.perm = torch.empty((B, H, n_rounds, L), **i32)
+        self.out = torch.empty(self.shape, dtype=self.tdtype, device=dev)
+        self.lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+        self.dqk = torch.empty(self.shape, dtype=torch.float32, device=dev)
+        self.dv = torch.empty(self.shape, dtype=torch.float32, device=dev)
+        self.ws_sort_bytes = _lib.lsh_sort_workspace_size(self.p)
+        self.ws_fwd_bytes = _lib.lsh_fwd_workspace_size(self.p)
+        self.ws_bwd_bytes = _lib.lsh_bwd_workspace_size(self.p)
+        if min(self.ws_sort_bytes, self.ws_fwd_bytes, self.ws_bwd_bytes) == 0 and B * H * L > 0:
+            raise _lib.LshError(1, "workspace size query (problem rejected)")
+        u8 = dict(dtype=torch.uint8, device=dev)
+        self.ws_sort = torch.empty(max(1, self.ws_sort_bytes), **u8)
+        self.ws_fwd = torch.empty(max(1, self.ws_fwd_bytes), **u8)
+        self.ws_bwd = torch.empty(max(1, self.ws_bwd_bytes), **u8)
+
+    def hash(self, qk, R, stream=None):
+        _lib.lsh_hash(self.p, qk, R, self.bucket, stream)
+        return self.bucket
+
+    def sort(self, bucket=None, stream=None):
+        _lib.lsh_sort(self.p, self.bucket if bucket is None else bucket, self.perm, self.ws_sort,
+                      self.ws_sort_bytes, stream)
+        return self.perm
+
+    def attend(self, qk, v, perm=None, stream=None):
+        _lib.lsh_attn_fwd(self.p, qk, v, self.perm if perm is None else perm, self.out, self.lse,
+                          self.ws_fwd, self.ws_fwd_bytes, stream)
+        return self.out, self.lse
+
+    def forward(self, qk, v, R, stream=None):
+        """hash -> sort -> chunk attention + round combine. Returns (out, lse)."""
+        self.hash(qk, R, stream)
+        self.sort(None, stream)
+        return self.attend(qk, v, None, stream)
+
+    def backward(self, qk, v, dout, perm=None, stream=None):
+        """Gradients of sum(out * dout) w.r.t. qk and v (float32)."""
+        _lib.lsh_attn_bwd(self.p, qk, v, self.perm if perm is None else perm, self.out, self.lse,
+                          dout, self.dqk, self.dv, self.ws_bwd, self.ws_bwd_bytes, stream)
+        return self.dqk, self.dv
+
+
+class _LSHAttentionFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, qk, v, R, runner: LSHAttention):
+        qk = qk.contiguous()
+        v = v.contiguous()
+        out, lse = runner.forward(qk, v, R.contiguous())
+        ctx.runner = runner
+        ctx.save_for_backward(qk, v)
+        return out.clone(), lse.clone()
+
+    @staticmethod
+    def backward(ctx, dout, dlse):
+        qk, v = ctx.saved_tensors
+        dqk, dv = ctx.runner.backward(qk, v, dout.contiguous().to(qk.dtype))
+        return dqk.to(qk.dtype), dv.to(v.dtype), None, None
+
+
+def lsh_attention(qk: torch.Tensor, v: torch.Tensor, R: torch.Tensor, n_buckets: int, chunk: int,
+                  causal: bool = True, scale: Optional[float] = None):
+    """Autograd-aware LSH self-attention. qk, v: [B,H,L,d]; R: [n_rounds,d,n_buckets/2].
+
+    Returns (out [B,H,L,d], lse [B,H,L]); gradients flow to qk and v (the
+    gradient of lse is not propagated).
+    """
+    B, H, L, d = qk.shape
+    dtype = {torch.float32: "f32", torch.bfloat16: "bf16"}[qk.dtype]
+    runner = LSHAttention(B, H, L, n_buckets, R.shape[0], chunk, causal, dtype, d, scale,
+                          qk.device)
+    return _LSHAttentionFn.apply(qk, v, R, runner)

@@ -1,0 +1,435 @@
+// Chunked LSH attention on CUDA cores: per-round forward, round combine,
+// and the recomputing backward pass. Serves float32 inputs and every shape.
+//
+// "Reformer: The Efficient Transformer" (research.elamur.ai summary page):
+//  - Key points, "LSH attention": after sorting, each chunk of m positions
+//    attends to itself and the chunk before it;
+//  - Key points, "Shared-QK Transformer": keys are the queries; a token does
+//    not attend to itself unless it has no other valid target;
+//  - Key points, "Number of hash rounds": several rounds; here they are
+//    combined by a softmax over their per-round log-sum-exps;
+//  - Summary: activations are recomputed instead of stored, which is what the
+//    backward does with the attention weights.
+//
+// Block = 64 sorted query slots of one (batch, head, round) segment; the
+// key window [max(0,(c-1)m), (c+1)m) is walked in tiles of 64 keys.
+// Thread (ty, tx) of a 16x16 grid owns rows ty*4+i and columns tx+16j.
+#include "common.cuh"
+#include "internal.h"
+
+namespace lsh {
+namespace {
+
+constexpr int kQ = 64;    // query rows per block
+constexpr int kK = 64;    // keys per tile
+constexpr int kP = kD + 1;  // padded shared-memory row (floats)
+
+// Reads perm[i]; an id outside [0, L) is recorded in the status word and
+// replaced by 0 so that no gather leaves the tensor.
+__device__ __forceinline__ int checked_pos(const int32_t* pr, int i, int L, int* status) {
+  int q = pr[i];
+  if ((unsigned)q >= (unsigned)L) {
+    if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
+    q = 0;
+  }
+  return q;
+}
+
+template <typename T>
+__device__ __forceinline__ void load_rows(float (*dst)[kP], const T* __restrict__ base,
+                                          const int* pos, int tid) {
+  for (int e = tid; e < kK * (kD / 4); e += 256) {
+    int row = e >> 4, c4 = (e & 15) * 4;
+    float4 f = load4(base + (int64_t)pos[row] * kD + c4);
+    dst[row][c4] = f.x; dst[row][c4 + 1] = f.y; dst[row][c4 + 2] = f.z; dst[row][c4 + 3] = f.w;
+  }
+}
+
+// Per-round forward. Writes o_r (normalised) and lse_r in original order.
+template <typename T>
+__global__ void __launch_bounds__(256)
+fwd_round_kernel(const T* __restrict__ qk, const T* __restrict__ v, const int32_t* __restrict__ perm,
+                 float* __restrict__ opart, float* __restrict__ lsepart, int L, int m,
+                 int n_rounds, int64_t N, int causal, float scale_log2, int* status) {
+  extern __shared__ float smem[];
+  float(*Qs)[kP] = reinterpret_cast<float(*)[kP]>(smem);
+  float(*Ks)[kP] = Qs + kQ;
+  float(*Vs)[kP] = Ks + kK;
+  float(*Ps)[kP] = Vs + kK;
+  int* qpos = reinterpret_cast<int*>(Ps + kQ);
+  int* kpos = qpos + kQ;
+
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int qblocks = L / kQ;
+  const int qb = blockIdx.x % qblocks;
+  const int64_t seg = blockIdx.x / qblocks;
+  const int r = (int)(seg % n_rounds);
+  const int64_t bh = seg / n_rounds;
+  const int32_t* pr = perm + seg * L;
+  const T* X = qk + bh * L * kD;
+  const T* Vb = v + bh * L * kD;
+  const int t0 = qb * kQ, c = t0 / m;
+  const int k_lo = max(0, (c - 1) * m), k_hi = (c + 1) * m;
+
+  if (tid < kQ) qpos[tid] = checked_pos(pr, t0 + tid, L, status);
+  __syncthreads();
+  load_rows(Qs, X, qpos, tid);
+  int myq[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) myq[i] = qpos[ty * 4 + i];
+
+  float mrow[4], lrow[4], acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    mrow[i] = -INFINITY; lrow[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  }
+
+  for (int kt = k_lo; kt < k_hi; kt += kK) {
+    __syncthreads();
+    if (tid < kK) kpos[tid] = checked_pos(pr, kt + tid, L, status);
+    __syncthreads();
+    load_rows(Ks, X, kpos, tid);
+    load_rows(Vs, Vb, kpos, tid);
+    __syncthreads();
+    float s[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s[i][j] = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < kD; ++k) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = Qs[ty * 4 + i][k];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Ks[tx + 16 * j][k];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) s[i][j] = fmaf(a[i], b[j], s[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        int kp = kpos[tx + 16 * j];
+        bool ok = (kp != myq[i]) && (!causal || kp < myq[i]);
+        s[i][j] = ok ? s[i][j] * scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, s[i][j]);
+      }
+      tmax = warp_max16(tmax);
+      float mnew = fmaxf(mrow[i], tmax);
+      float msafe = (mnew == -INFINITY) ? 0.f : mnew;
+      float alpha = exp2f(mrow[i] - msafe);
+      float rs = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float pv = exp2f(s[i][j] - msafe);
+        Ps[ty * 4 + i][tx + 16 * j] = pv;
+        rs += pv;
+      }
+      rs = warp_sum16(rs);
+      lrow[i] = lrow[i] * alpha + rs;
+      mrow[i] = mnew;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] *= alpha;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < kK; ++k) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = Ps[ty * 4 + i][k];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Vs[k][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t row = (int64_t)r * N + bh * L + myq[i];
+    const bool has = lrow[i] > 0.f;
+    const float inv = has ? 1.f / lrow[i] : 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) opart[row * kD + tx + 16 * j] = acc[i][j] * inv;
+    if (tx == 0) lsepart[row] = has ? (mrow[i] + log2f(lrow[i])) * kLn2 : -INFINITY;
+  }
+}
+
+// Round combine in original order; 16 threads per token, 4 columns each.
+template <typename T>
+__global__ void __launch_bounds__(256)
+combine_kernel(const float* __restrict__ opart, const float* __restrict__ lsepart,
+               const T* __restrict__ v, T* __restrict__ out, float* __restrict__ lse, int64_t N,
+               int n_rounds) {
+  const int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
+  const int c4 = (threadIdx.x & 15) * 4;
+  if (tok >= N) return;
+  float mx = -INFINITY;
+  for (int r = 0; r < n_rounds; ++r) mx = fmaxf(mx, lsepart[(int64_t)r * N + tok]);
+  if (mx == -INFINITY) {
+    store4(out + tok * kD + c4, load4(v + tok * kD + c4));
+    if (c4 == 0) lse[tok] = -INFINITY;
+    return;
+  }
+  float tot = 0.f;
+  for (int r = 0; r < n_rounds; ++r) tot += expf(lsepart[(int64_t)r * N + tok] - mx);
+  const float LSE = mx + logf(tot);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int r = 0; r < n_rounds; ++r) {
+    float l = lsepart[(int64_t)r * N + tok];
+    if (l == -INFINITY) continue;
+    float w = expf(l - LSE);
+    float4 o = load4(opart + ((int64_t)r * N + tok) * kD + c4);
+    acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
+  }
+  store4(out + tok * kD + c4, acc);
+  if (c4 == 0) lse[tok] = LSE;
+}
+
+// D_i = dout_i . out_i; zero dqk; dv = dout for self-attending rows, else 0.
+template <typename T>
+__global__ void __launch_bounds__(256)
+bwd_prep_kernel(const T* __restrict__ out, const T* __restrict__ dout, const float* __restrict__ lse,
+                float* __restrict__ D, float* __restrict__ dqk, float* __restrict__ dv, int64_t N) {
+  const int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
+  const int c4 = (threadIdx.x & 15) * 4;
+  const bool live = tok < N;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f), g = o;
+  if (live) { o = load4(out + tok * kD + c4); g = load4(dout + tok * kD + c4); }
+  float d = warp_sum16(o.x * g.x + o.y * g.y + o.z * g.z + o.w * g.w);
+  if (!live) return;
+  if (c4 == 0) D[tok] = d;
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  store4(dqk + tok * kD + c4, z);
+  store4(dv + tok * kD + c4, lse[tok] == -INFINITY ? g : z);
+}
+
+// Backward for one block of 64 query slots: recompute P from the final LSE,
+// dS = P (dO.v - D); query-side dqk in registers, key-side dqk/dv by atomics.
+template <typename T>
+__global__ void __launch_bounds__(256)
+bwd_round_kernel(const T* __restrict__ qk, const T* __restrict__ v, const T* __restrict__ dout,
+                 const int32_t* __restrict__ perm, const float* __restrict__ lse,
+                 const float* __restrict__ D, float* __restrict__ dqk, float* __restrict__ dv,
+                 int L, int m, int n_rounds, int causal, float scale, float scale_log2,
+                 int* status) {
+  extern __shared__ float smem[];
+  float(*Qs)[kP] = reinterpret_cast<float(*)[kP]>(smem);
+  float(*Gs)[kP] = Qs + kQ;
+  float(*Ks)[kP] = Gs + kQ;
+  float(*Vs)[kP] = Ks + kK;
+  float(*Ps)[kP] = Vs + kK;
+  float(*Ss)[kP] = Ps + kQ;
+  int* qpos = reinterpret_cast<int*>(Ss + kQ);
+  int* kpos = qpos + kQ;
+  float* qlse = reinterpret_cast<float*>(kpos + kK);
+  float* qD = qlse + kQ;
+
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int qblocks = L / kQ;
+  const int qb = blockIdx.x % qblocks;
+  const int64_t seg = blockIdx.x / qblocks;
+  const int64_t bh = seg / n_rounds;
+  const int32_t* pr = perm + seg * L;
+  const T* X = qk + bh * L * kD;
+  const T* Vb = v + bh * L * kD;
+  const T* Gb = dout + bh * L * kD;
+  float* dX = dqk + bh * L * kD;
+  float* dV = dv + bh * L * kD;
+  const int t0 = qb * kQ, c = t0 / m;
+  const int k_lo = max(0, (c - 1) * m), k_hi = (c + 1) * m;
+
+  if (tid < kQ) {
+    int q = checked_pos(pr, t0 + tid, L, status);
+    qpos[tid] = q;
+    qlse[tid] = lse[bh * L + q] * kLog2e;
+    qD[tid] = D[bh * L + q];
+  }
+  __syncthreads();
+  load_rows(Qs, X, qpos, tid);
+  load_rows(Gs, Gb, qpos, tid);
+  int myq[4];
+  float ml[4], md[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) { myq[i] = qpos[ty * 4 + i]; ml[i] = qlse[ty * 4 + i]; md[i] = qD[ty * 4 + i]; }
+  float dq[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dq[i][j] = 0.f;
+
+  for (int kt = k_lo; kt < k_hi; kt += kK) {
+    __syncthreads();
+    if (tid < kK) kpos[tid] = checked_pos(pr, kt + tid, L, status);
+    __syncthreads();
+    load_rows(Ks, X, kpos, tid);
+    load_rows(Vs, Vb, kpos, tid);
+    __syncthreads();
+    float s[4][4], dp[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) { s[i][j] = 0.f; dp[i][j] = 0.f; }
+#pragma unroll 4
+    for (int k = 0; k < kD; ++k) {
+      float a[4], g[4], b[4], w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { a[i] = Qs[ty * 4 + i][k]; g[i] = Gs[ty * 4 + i][k]; }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) { b[j] = Ks[tx + 16 * j][k]; w[j] = Vs[tx + 16 * j][k]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          s[i][j] = fmaf(a[i], b[j], s[i][j]);
+          dp[i][j] = fmaf(g[i], w[j], dp[i][j]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        int kp = kpos[tx + 16 * j];
+        bool ok = (kp != myq[i]) && (!causal || kp < myq[i]) && (ml[i] != -INFINITY);
+        float pv = ok ? exp2f(s[i][j] * scale_log2 - ml[i]) : 0.f;
+        Ps[ty * 4 + i][tx + 16 * j] = pv;
+        Ss[ty * 4 + i][tx + 16 * j] = pv * (dp[i][j] - md[i]);
+      }
+    __syncthreads();
+    // query side: dq += dS K
+#pragma unroll 4
+    for (int k = 0; k < kK; ++k) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = Ss[ty * 4 + i][k];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Ks[k][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dq[i][j] = fmaf(a[i], b[j], dq[i][j]);
+    }
+    // key side: dk = dS^T Q, dvv = P^T dO, for keys ty*4+i
+    float dk[4][4], dvv[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) { dk[i][j] = 0.f; dvv[i][j] = 0.f; }
+#pragma unroll 4
+    for (int q = 0; q < kQ; ++q) {
+      float sa[4], pa[4], qb4[4], gb4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { sa[i] = Ss[q][ty * 4 + i]; pa[i] = Ps[q][ty * 4 + i]; }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) { qb4[j] = Qs[q][tx + 16 * j]; gb4[j] = Gs[q][tx + 16 * j]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          dk[i][j] = fmaf(sa[i], qb4[j], dk[i][j]);
+          dvv[i][j] = fmaf(pa[i], gb4[j], dvv[i][j]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t krow = (int64_t)kpos[ty * 4 + i] * kD;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        atomicAdd(dX + krow + tx + 16 * j, scale * dk[i][j]);
+        atomicAdd(dV + krow + tx + 16 * j, dvv[i][j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t qrow = (int64_t)myq[i] * kD;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) atomicAdd(dX + qrow + tx + 16 * j, scale * dq[i][j]);
+  }
+}
+
+constexpr size_t kFwdSmem = (size_t)(2 * kQ + 2 * kK) * kP * 4 + (kQ + kK) * 4;
+constexpr size_t kBwdSmem = (size_t)(4 * kQ + 2 * kK) * kP * 4 + (kQ + kK) * 4 + 2 * kQ * 4;
+
+template <typename T>
+cudaError_t fwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* perm, T* out,
+                  float* lse, const FwdWs& ws, int* status, cudaStream_t s) {
+  const int64_t N = (int64_t)p.B * p.H * p.L;
+  const int64_t blocks = (int64_t)p.B * p.H * p.n_rounds * (p.L / kQ);
+  cudaError_t e = cudaFuncSetAttribute(fwd_round_kernel<T>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdSmem);
+  if (e != cudaSuccess) return e;
+  fwd_round_kernel<T><<<(unsigned)blocks, 256, kFwdSmem, s>>>(
+      qk, v, perm, ws.opart, ws.lsepart, p.L, p.chunk, p.n_rounds, N, p.causal,
+      p.scale * kLog2e, status);
+  combine_kernel<T><<<(unsigned)((N * 16 + 255) / 256), 256, 0, s>>>(ws.opart, ws.lsepart, v, out,
+                                                                     lse, N, p.n_rounds);
+  note_launch(2);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t bwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* perm, const T* out,
+                  const float* lse, const T* dout, float* dqk, float* dv, float* D, int* status,
+                  cudaStream_t s) {
+  const int64_t N = (int64_t)p.B * p.H * p.L;
+  const int64_t blocks = (int64_t)p.B * p.H * p.n_rounds * (p.L / kQ);
+  cudaError_t e = cudaFuncSetAttribute(bwd_round_kernel<T>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem);
+  if (e != cudaSuccess) return e;
+  bwd_prep_kernel<T><<<(unsigned)((N * 16 + 255) / 256), 256, 0, s>>>(out, dout, lse, D, dqk, dv, N);
+  bwd_round_kernel<T><<<(unsigned)blocks, 256, kBwdSmem, s>>>(
+      qk, v, dout, perm, lse, D, dqk, dv, p.L, p.chunk, p.n_rounds, p.causal, p.scale,
+      p.scale * kLog2e, status);
+  note_launch(2);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t fwd_ws_bytes(const lsh_problem& p) {
+  const size_t N = (size_t)p.B * p.H * p.L;
+  return align_up((size_t)p.n_rounds * N * kD * 4, 256) + align_up((size_t)p.n_rounds * N * 4, 256);
+}
+
+FwdWs fwd_ws_carve(const lsh_problem& p, void* ws) {
+  const size_t N = (size_t)p.B * p.H * p.L;
+  FwdWs w;
+  w.opart = (float*)ws;
+  w.lsepart = (float*)((char*)ws + align_up((size_t)p.n_rounds * N * kD * 4, 256));
+  return w;
+}
+
+cudaError_t launch_attn_fwd(const lsh_problem& p, const void* qk, const void* v,
+                            const int32_t* perm, void* out, float* lse, const FwdWs& ws,
+                            int* status, cudaStream_t s) {
+  if (p.dtype == LSH_BF16)
+    return fwd_t(p, (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, perm, (__nv_bfloat16*)out,
+                 lse, ws, status, s);
+  return fwd_t(p, (const float*)qk, (const float*)v, perm, (float*)out, lse, ws, status, s);
+}
+
+size_t bwd_ws_bytes(const lsh_problem& p) {
+  return align_up((size_t)p.B * p.H * p.L * 4, 256);
+}
+
+cudaError_t launch_attn_bwd(const lsh_problem& p, const void* qk, const void* v,
+                            const int32_t* perm, const void* out, const float* lse,
+                            const void* dout, float* dqk, float* dv, void* ws, int* status,
+                            cudaStream_t s) {
+  float* D = (float*)ws;
+  if (p.dtype == LSH_BF16)
+    return bwd_t(p, (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, perm,
+                 (const __nv_bfloat16*)out, lse, (const __nv_bfloat16*)dout, dqk, dv, D, status, s);
+  return bwd_t(p, (const float*)qk, (const float*)v, perm, (const float*)out, lse,
+               (const float*)dout, dqk, dv, D, status, s);
+}
+
+}  // namespace lsh

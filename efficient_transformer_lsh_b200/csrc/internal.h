@@ -1,0 +1,59 @@
+// Host-side interface between the C ABI (lsh_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "lsh.h"
+
+namespace lsh {
+
+constexpr int kDHead = 64;  // the only head size the kernels support
+
+// Counts one kernel launch (for lsh_launch_count()).
+void note_launch(int n = 1);
+
+// Device status word of the current device (LSH_OK until a kernel records a
+// timeout or an index check); nullptr if it cannot be resolved.
+int* device_status_word();
+
+// ---- hashing ----
+cudaError_t launch_hash_simt(const lsh_problem& p, const void* qk, const void* R,
+                             int32_t* bucket, cudaStream_t s);
+// tcgen05 path (bf16 inputs); returns cudaErrorNotSupported when the shape
+// does not suit it, so the caller can choose the SIMT kernel instead.
+cudaError_t launch_hash_tc(const lsh_problem& p, const void* qk, const void* R,
+                           int32_t* bucket, int* status, cudaStream_t s);
+
+// ---- sorting ----
+struct SortWs {
+  uint32_t* sorted;   // [S * L] tile-sorted packed keys
+  int32_t* counts;    // [S * n_buckets * tiles]
+  int32_t* base;      // [S * n_buckets]
+};
+size_t sort_ws_bytes(const lsh_problem& p);
+SortWs sort_ws_carve(const lsh_problem& p, void* ws);
+cudaError_t launch_sort(const lsh_problem& p, const int32_t* bucket, int32_t* perm,
+                        const SortWs& ws, int* status, cudaStream_t s);
+
+// ---- attention ----
+struct FwdWs {
+  float* opart;    // [n_rounds, B*H*L, d] per-round outputs, original order
+  float* lsepart;  // [n_rounds, B*H*L] per-round log-sum-exps
+};
+size_t fwd_ws_bytes(const lsh_problem& p);
+FwdWs fwd_ws_carve(const lsh_problem& p, void* ws);
+cudaError_t launch_attn_fwd(const lsh_problem& p, const void* qk, const void* v,
+                            const int32_t* perm, void* out, float* lse, const FwdWs& ws,
+                            int* status, cudaStream_t s);
+
+size_t bwd_ws_bytes(const lsh_problem& p);
+cudaError_t launch_attn_bwd(const lsh_problem& p, const void* qk, const void* v,
+                            const int32_t* perm, const void* out, const float* lse,
+                            const void* dout, float* dqk, float* dv, void* ws,
+                            int* status, cudaStream_t s);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace lsh

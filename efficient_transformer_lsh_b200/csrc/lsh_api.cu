@@ -1,0 +1,167 @@
+// C ABI of the LSH-attention library: argument checks, workspace sizing,
+// dispatch to the kernels, and the device status word.
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+#include "internal.h"
+
+namespace lsh {
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+// Device status word: kernels record LSH_ERR_TIMEOUT / LSH_ERR_DEVICE_CHECK
+// here instead of trapping, so the context stays usable.
+__device__ int g_status_word;
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {};
+std::mutex g_status_mu;
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+lsh_status check_problem(const lsh_problem* p) {
+  if (!p) return LSH_ERR_INVALID_ARG;
+  if (p->B < 0 || p->H < 0 || p->L < 0 || p->d <= 0) return LSH_ERR_INVALID_ARG;
+  if (p->n_buckets < 2 || p->n_buckets % 2 != 0 || p->n_buckets > 65536) return LSH_ERR_INVALID_ARG;
+  if (p->n_rounds < 1 || p->n_rounds > 64) return LSH_ERR_INVALID_ARG;
+  if (p->chunk <= 0) return LSH_ERR_INVALID_ARG;
+  if (p->L % p->chunk != 0) return LSH_ERR_INVALID_ARG;
+  if (p->causal != 0 && p->causal != 1) return LSH_ERR_INVALID_ARG;
+  if (!std::isfinite(p->scale)) return LSH_ERR_INVALID_ARG;
+  if (p->dtype != LSH_F32 && p->dtype != LSH_BF16) return LSH_ERR_INVALID_ARG;
+  if (p->d != kDHead) return LSH_ERR_UNSUPPORTED;
+  if (p->chunk % 64 != 0) return LSH_ERR_UNSUPPORTED;
+  // int32 positions, and per-round index spaces addressed in 32 bits
+  const int64_t rows = (int64_t)p->B * p->H * p->L;
+  if ((int64_t)p->n_rounds * rows > (int64_t)INT32_MAX) return LSH_ERR_UNSUPPORTED;
+  if ((int64_t)p->B * p->H * p->n_rounds * (p->L / 64) > (int64_t)INT32_MAX)
+    return LSH_ERR_UNSUPPORTED;
+  return LSH_OK;
+}
+
+bool empty(const lsh_problem* p) { return (int64_t)p->B * p->H * p->L == 0; }
+
+lsh_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LSH_OK : LSH_ERR_CUDA; }
+
+}  // namespace
+
+void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+int* device_status_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_status_word) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = (int*)ptr;
+  }
+  return g_status_ptr[dev];
+}
+
+}  // namespace lsh
+
+using namespace lsh;
+
+extern "C" {
+
+lsh_status lsh_hash(const lsh_problem* p, const void* qk, const void* R, int32_t* bucket,
+                    lsh_stream_t stream) {
+  lsh_status st = check_problem(p);
+  if (st != LSH_OK) return st;
+  if (empty(p)) return LSH_OK;
+  if (!qk || !R || !bucket) return LSH_ERR_INVALID_ARG;
+  if (!aligned(qk, 16)) return LSH_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (p->dtype == LSH_BF16) {
+    int* status = device_status_word();
+    cudaError_t e = launch_hash_tc(*p, qk, R, bucket, status, s);
+    if (e != cudaErrorNotSupported) return cuda_status(e);
+  }
+  return cuda_status(launch_hash_simt(*p, qk, R, bucket, s));
+}
+
+size_t lsh_sort_workspace_size(const lsh_problem* p) {
+  if (check_problem(p) != LSH_OK) return 0;
+  return sort_ws_bytes(*p);
+}
+
+lsh_status lsh_sort(const lsh_problem* p, const int32_t* bucket, int32_t* perm, void* ws,
+                    size_t ws_bytes, lsh_stream_t stream) {
+  lsh_status st = check_problem(p);
+  if (st != LSH_OK) return st;
+  if (empty(p)) return LSH_OK;
+  if (!bucket || !perm) return LSH_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < sort_ws_bytes(*p) || !aligned(ws, 256)) return LSH_ERR_WORKSPACE;
+  return cuda_status(launch_sort(*p, bucket, perm, sort_ws_carve(*p, ws), device_status_word(),
+                                 (cudaStream_t)stream));
+}
+
+size_t lsh_fwd_workspace_size(const lsh_problem* p) {
+  if (check_problem(p) != LSH_OK) return 0;
+  return fwd_ws_bytes(*p);
+}
+
+lsh_status lsh_attn_fwd(const lsh_problem* p, const void* qk, const void* v, const int32_t* perm,
+                        void* out, float* lse, void* ws, size_t ws_bytes, lsh_stream_t stream) {
+  lsh_status st = check_problem(p);
+  if (st != LSH_OK) return st;
+  if (empty(p)) return LSH_OK;
+  if (!qk || !v || !perm || !out || !lse) return LSH_ERR_INVALID_ARG;
+  if (!aligned(qk, 16) || !aligned(v, 16) || !aligned(out, 16)) return LSH_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < fwd_ws_bytes(*p) || !aligned(ws, 256)) return LSH_ERR_WORKSPACE;
+  return cuda_status(launch_attn_fwd(*p, qk, v, perm, out, lse, fwd_ws_carve(*p, ws),
+                                     device_status_word(), (cudaStream_t)stream));
+}
+
+size_t lsh_bwd_workspace_size(const lsh_problem* p) {
+  if (check_problem(p) != LSH_OK) return 0;
+  return bwd_ws_bytes(*p);
+}
+
+lsh_status lsh_attn_bwd(const lsh_problem* p, const void* qk, const void* v, const int32_t* perm,
+                        const void* out, const float* lse, const void* dout, float* dqk,
+                        float* dv, void* ws, size_t ws_bytes, lsh_stream_t stream) {
+  lsh_status st = check_problem(p);
+  if (st != LSH_OK) return st;
+  if (empty(p)) return LSH_OK;
+  if (!qk || !v || !perm || !out || !lse || !dout || !dqk || !dv) return LSH_ERR_INVALID_ARG;
+  if (!aligned(qk, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(dout, 16) ||
+      !aligned(dqk, 16) || !aligned(dv, 16))
+    return LSH_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < bwd_ws_bytes(*p) || !aligned(ws, 256)) return LSH_ERR_WORKSPACE;
+  return cuda_status(launch_attn_bwd(*p, qk, v, perm, out, lse, dout, dqk, dv, ws,
+                                     device_status_word(), (cudaStream_t)stream));
+}
+
+lsh_status lsh_device_status(lsh_stream_t stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return LSH_ERR_CUDA;
+  int* w = device_status_word();
+  if (!w) return LSH_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return LSH_ERR_CUDA;
+  if (v != 0) {
+    int z = 0;
+    if (cudaMemcpy(w, &z, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return LSH_ERR_CUDA;
+  }
+  return (lsh_status)v;
+}
+
+const char* lsh_status_string(lsh_status s) {
+  switch (s) {
+    case LSH_OK: return "ok";
+    case LSH_ERR_INVALID_ARG: return "invalid argument";
+    case LSH_ERR_UNSUPPORTED: return "unsupported problem (d must be 64, chunk a multiple of 64)";
+    case LSH_ERR_WORKSPACE: return "workspace missing, too small or not 256-byte aligned";
+    case LSH_ERR_CUDA: return "CUDA runtime error";
+    case LSH_ERR_TIMEOUT: return "a kernel timed out waiting on a barrier";
+    case LSH_ERR_DEVICE_CHECK: return "a kernel found an out-of-range index";
+  }
+  return "unknown status";
+}
+
+uint64_t lsh_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

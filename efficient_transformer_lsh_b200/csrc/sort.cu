@@ -1,0 +1,218 @@
+// Stable sort of positions by bucket, one segment per (batch, head, round).
+//
+// "Reformer: The Efficient Transformer" (research.elamur.ai summary page),
+// Summary and Key points "LSH attention": positions are sorted by bucket
+// before chunking. Sorting stably by bucket is sorting by the packed key
+// (round, bucket, position), because positions arrive in increasing order.
+//
+// Counting sort in four passes over tiles of kTile positions:
+//   1. tile_sort: each tile sorts packed keys (bucket << 12 | local index) in
+//      shared memory (bitonic network), stores them, and records how many
+//      positions of each bucket it holds: counts[seg][bucket][tile];
+//   2. row_scan: for every (seg, bucket), exclusive scan over tiles, plus the
+//      bucket total;
+//   3. bucket_scan: for every seg, exclusive scan of bucket totals;
+//   4. scatter: slot = base[seg][b] + counts[seg][b][tile] + rank within the
+//      tile's run of bucket b; perm[seg][slot] = position.
+// The packed local index makes every tile's order stable, and tiles are
+// placed in position order, so the whole sort is stable.
+#include "common.cuh"
+#include "internal.h"
+
+namespace lsh {
+namespace {
+
+constexpr int kTile = 4096;        // positions per tile (12-bit local index)
+constexpr int kTileThreads = 1024;
+
+__device__ __forceinline__ void bitonic_sort_smem(uint32_t* s) {
+  const int tid = threadIdx.x;
+  for (int k = 2; k <= kTile; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int e = tid; e < kTile / 2; e += kTileThreads) {
+        int i = (e / j) * 2 * j + (e % j);
+        int ip = i + j;
+        bool up = (i & k) == 0;
+        uint32_t a = s[i], b = s[ip];
+        if ((a > b) == up) { s[i] = b; s[ip] = a; }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// First index in the sorted tile whose bucket is >= b.
+__device__ __forceinline__ int lower_bound_bucket(const uint32_t* s, uint32_t b) {
+  uint32_t key = b << 12;
+  int lo = 0, hi = kTile;
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (s[mid] < key) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(kTileThreads)
+tile_sort_kernel(const int32_t* __restrict__ bucket, uint32_t* __restrict__ sorted,
+                 int32_t* __restrict__ counts, int L, int n_buckets, int tiles, int* status) {
+  __shared__ uint32_t s[kTile];
+  const int tile = blockIdx.x % tiles;
+  const int64_t seg = blockIdx.x / tiles;
+  const int64_t p0 = (int64_t)tile * kTile;
+  const int n = min(kTile, (int)(L - p0));
+  const int32_t* src = bucket + seg * L + p0;
+  for (int i = threadIdx.x; i < kTile; i += kTileThreads) {
+    uint32_t key = 0xffffffffu;
+    if (i < n) {
+      uint32_t b = (uint32_t)src[i];
+      if (b >= (uint32_t)n_buckets) {   // out-of-range id: flag it, keep memory safe
+        if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
+        b = (uint32_t)n_buckets - 1;
+      }
+      key = (b << 12) | (uint32_t)i;
+    }
+    s[i] = key;
+  }
+  __syncthreads();
+  bitonic_sort_smem(s);
+  uint32_t* dst = sorted + seg * L + p0;
+  for (int i = threadIdx.x; i < n; i += kTileThreads) {
+    uint32_t key = s[i];
+    dst[i] = key;
+    uint32_t b = key >> 12;
+    bool last = (i == n - 1) || ((s[i + 1] >> 12) != b);
+    if (last) {
+      int first = lower_bound_bucket(s, b);
+      counts[(seg * n_buckets + b) * tiles + tile] = i - first + 1;
+    }
+  }
+}
+
+// One warp per (seg, bucket): exclusive scan of counts over tiles; writes the
+// bucket total to base[seg][bucket].
+__global__ void row_scan_kernel(int32_t* __restrict__ counts, int32_t* __restrict__ base,
+                                int64_t rows, int tiles) {
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  int32_t* c = counts + row * tiles;
+  int carry = 0;
+  for (int t0 = 0; t0 < tiles; t0 += 32) {
+    int t = t0 + lane;
+    int v = (t < tiles) ? c[t] : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (t < tiles) c[t] = carry + x - v;
+    carry += __shfl_sync(0xffffffffu, x, 31);
+  }
+  if (lane == 0) base[row] = carry;
+}
+
+// One block per segment: exclusive scan of the bucket totals, in place.
+__global__ void __launch_bounds__(1024)
+bucket_scan_kernel(int32_t* __restrict__ base, int n_buckets) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry_s;
+  int32_t* b = base + (int64_t)blockIdx.x * n_buckets;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) carry_s = 0;
+  __syncthreads();
+  for (int i0 = 0; i0 < n_buckets; i0 += 1024) {
+    int i = i0 + threadIdx.x;
+    int v = (i < n_buckets) ? b[i] : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_tot[lane];
+      int wx = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, wx, o);
+        if (lane >= o) wx += y;
+      }
+      warp_tot[lane] = wx - w;   // exclusive prefix of warp totals
+    }
+    __syncthreads();
+    int carry = carry_s;
+    if (i < n_buckets) b[i] = carry + warp_tot[warp] + x - v;
+    __syncthreads();
+    if (threadIdx.x == 1023) carry_s = carry + warp_tot[31] + x;
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(kTileThreads)
+scatter_kernel(const uint32_t* __restrict__ sorted, const int32_t* __restrict__ counts,
+               const int32_t* __restrict__ base, int32_t* __restrict__ perm, int L,
+               int n_buckets, int tiles) {
+  __shared__ uint32_t s[kTile];
+  const int tile = blockIdx.x % tiles;
+  const int64_t seg = blockIdx.x / tiles;
+  const int64_t p0 = (int64_t)tile * kTile;
+  const int n = min(kTile, (int)(L - p0));
+  const uint32_t* src = sorted + seg * L + p0;
+  for (int i = threadIdx.x; i < kTile; i += kTileThreads) s[i] = (i < n) ? src[i] : 0xffffffffu;
+  __syncthreads();
+  int32_t* out = perm + seg * L;
+  for (int i = threadIdx.x; i < n; i += kTileThreads) {
+    uint32_t key = s[i];
+    uint32_t b = key >> 12;
+    int first = lower_bound_bucket(s, b);
+    int64_t row = seg * n_buckets + b;
+    int slot = base[row] + counts[row * tiles + tile] + (i - first);
+    out[slot] = (int32_t)(p0 + (key & 0xfffu));
+  }
+}
+
+}  // namespace
+
+size_t sort_ws_bytes(const lsh_problem& p) {
+  const int64_t S = (int64_t)p.B * p.H * p.n_rounds;
+  const int64_t tiles = (p.L + kTile - 1) / kTile;
+  size_t b = align_up((size_t)S * p.L * 4, 256);
+  b += align_up((size_t)S * p.n_buckets * tiles * 4, 256);
+  b += align_up((size_t)S * p.n_buckets * 4, 256);
+  return b;
+}
+
+SortWs sort_ws_carve(const lsh_problem& p, void* ws) {
+  const int64_t S = (int64_t)p.B * p.H * p.n_rounds;
+  const int64_t tiles = (p.L + kTile - 1) / kTile;
+  char* c = (char*)ws;
+  SortWs w;
+  w.sorted = (uint32_t*)c;
+  c += align_up((size_t)S * p.L * 4, 256);
+  w.counts = (int32_t*)c;
+  c += align_up((size_t)S * p.n_buckets * tiles * 4, 256);
+  w.base = (int32_t*)c;
+  return w;
+}
+
+cudaError_t launch_sort(const lsh_problem& p, const int32_t* bucket, int32_t* perm,
+                        const SortWs& ws, int* status, cudaStream_t s) {
+  const int64_t S = (int64_t)p.B * p.H * p.n_rounds;
+  const int tiles = (p.L + kTile - 1) / kTile;
+  const int64_t rows = S * p.n_buckets;
+  cudaError_t e = cudaMemsetAsync(ws.counts, 0, (size_t)rows * tiles * 4, s);
+  if (e != cudaSuccess) return e;
+  tile_sort_kernel<<<(unsigned)(S * tiles), kTileThreads, 0, s>>>(bucket, ws.sorted, ws.counts, p.L,
+                                                               p.n_buckets, tiles, status);
+  row_scan_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(ws.counts, ws.base, rows, tiles);
+  bucket_scan_kernel<<<(unsigned)S, 1024, 0, s>>>(ws.base, p.n_buckets);
+  scatter_kernel<<<(unsigned)(S * tiles), kTileThreads, 0, s>>>(ws.sorted, ws.counts, ws.base, perm,
+                                                             p.L, p.n_buckets, tiles);
+  note_launch(4);
+  return cudaGetLastError();
+}
+
+}  // namespace lsh

@@ -1,0 +1,139 @@
+/*
+ * lsh.h — C ABI of the B200 (sm_100a) Reformer LSH self-attention library.
+ *
+ * The method (sources: "Reformer: The Efficient Transformer", research.elamur.ai
+ * summary page — Summary paragraph and Key points "LSH attention",
+ * "Shared-QK Transformer", "Number of hash rounds"):
+ *   1. queries and keys are one shared vector x per token (shared-QK);
+ *   2. each hash round r maps x to a bucket h_r(x) = argmax([x R_r ; -x R_r])
+ *      with a random matrix R_r;
+ *   3. positions are sorted by bucket, separately for every round;
+ *   4. each chunk of m sorted positions attends to itself and the chunk
+ *      before it; a token does not attend to itself unless it has no other
+ *      valid target;
+ *   5. the rounds' outputs are combined by a softmax over their per-round
+ *      log-sum-exps; the backward pass recomputes the attention weights.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor arguments are DEVICE pointers, contiguous, row-major, owned
+ *     and allocated by the caller. The library allocates no memory; scratch
+ *     space comes from the caller through (ws, ws_bytes), 256-byte aligned,
+ *     of at least the size the matching *_workspace_size() returns.
+ *   - Work is queued asynchronously on `stream` (NULL = legacy default
+ *     stream). Nothing synchronises unless stated.
+ *   - Arguments are checked on the host before anything is launched; a bad
+ *     argument returns LSH_ERR_INVALID_ARG / LSH_ERR_UNSUPPORTED /
+ *     LSH_ERR_WORKSPACE and launches nothing. A failed launch returns
+ *     LSH_ERR_CUDA. Kernels that wait on hardware barriers give up after a
+ *     bounded number of polls and record LSH_ERR_TIMEOUT in a device status
+ *     word, read by lsh_device_status(). No C++ exception crosses the ABI.
+ *   - Outputs are overwritten, never accumulated into.
+ *   - Shapes: B batch, H heads, L sequence length, d head size (64),
+ *     n_buckets (even), n_rounds hash rounds, chunk = m.
+ *     qk, v, out, dout: [B, H, L, d] in `dtype`;
+ *     R: [n_rounds, d, n_buckets/2] in `dtype`;
+ *     bucket, perm: [B, H, n_rounds, L] int32;
+ *     lse: [B, H, L] float32; dqk, dv: [B, H, L, d] float32.
+ *   - B*H*L == 0 is a valid empty problem: nothing is launched, LSH_OK.
+ */
+#ifndef LSH_H
+#define LSH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* lsh_stream_t;
+
+typedef enum {
+  LSH_OK = 0,
+  LSH_ERR_INVALID_ARG = 1,   /* null pointer, bad size or bad combination      */
+  LSH_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d != 64)       */
+  LSH_ERR_WORKSPACE = 3,     /* workspace missing, too small or misaligned     */
+  LSH_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed           */
+  LSH_ERR_TIMEOUT = 5,       /* a kernel gave up waiting on a barrier          */
+  LSH_ERR_DEVICE_CHECK = 6   /* a kernel found an out-of-range index           */
+} lsh_status;
+
+typedef enum { LSH_F32 = 0, LSH_BF16 = 1 } lsh_dtype;
+
+typedef struct {
+  int32_t B, H, L, d;
+  int32_t n_buckets;   /* even, 2 .. 65536                                     */
+  int32_t n_rounds;    /* 1 .. 64                                              */
+  int32_t chunk;       /* m: a multiple of 64 that divides L                  */
+  int32_t causal;      /* 0: every key in the window; 1: keys at earlier positions only */
+  float scale;         /* logit scale, usually 1/sqrt(d)                      */
+  int32_t dtype;       /* lsh_dtype of qk, v, R, out, dout                    */
+} lsh_problem;
+
+/*
+ * lsh_hash — step 2 (Key points, "LSH attention": h(x) = argmax([xR; -xR])).
+ *   bucket[b,h,r,i] = argmax over the n_buckets entries of [x R_r ; -x R_r],
+ *   x = qk[b,h,i,:], lowest index on exact ties, for every round r.
+ *   The contraction accumulates exact products in float32 (bf16 inputs
+ *   multiply exactly; float32 inputs use fused multiply-add).
+ */
+lsh_status lsh_hash(const lsh_problem* p, const void* qk, const void* R,
+                    int32_t* bucket, lsh_stream_t stream);
+
+/*
+ * lsh_sort — step 3 (Summary and Key points: positions "sorted by bucket").
+ *   For every (b,h,r): perm[b,h,r,t] = original position of sorted slot t,
+ *   where positions are sorted stably by bucket, i.e. by the packed key
+ *   (round, bucket, position). bucket values must lie in [0, n_buckets).
+ */
+size_t lsh_sort_workspace_size(const lsh_problem* p);
+lsh_status lsh_sort(const lsh_problem* p, const int32_t* bucket, int32_t* perm,
+                    void* ws, size_t ws_bytes, lsh_stream_t stream);
+
+/*
+ * lsh_attn_fwd — steps 4 and 5 (Key points "LSH attention" and
+ *   "Shared-QK Transformer"). For each round, the query in sorted slot t
+ *   (chunk c = t / m) attends to the keys in slots [max(0,(c-1)m), (c+1)m)
+ *   of the same round. Key j is valid for query i iff j != i and, when
+ *   causal, j < i (original positions). Logits are scale * x_i . x_j.
+ *   Per round: lse_r,i (or -inf with no valid key) and o_r,i; then
+ *   lse[i] = log sum_r exp(lse_r,i), out[i] = sum_r exp(lse_r,i - lse[i]) o_r,i.
+ *   A token with no valid key in any round attends to itself:
+ *   out[i] = v[i], lse[i] = -inf.
+ */
+size_t lsh_fwd_workspace_size(const lsh_problem* p);
+lsh_status lsh_attn_fwd(const lsh_problem* p, const void* qk, const void* v,
+                        const int32_t* perm, void* out, float* lse,
+                        void* ws, size_t ws_bytes, lsh_stream_t stream);
+
+/*
+ * lsh_attn_bwd — gradient of sum(out * dout) with respect to qk and v,
+ *   recomputing the attention weights P_ij = exp(s_ij - lse_i) instead of
+ *   storing them (the Reformer's recompute-instead-of-store principle,
+ *   Summary paragraph). D_i = dout_i . out_i; dS = P (dout_i . v_j - D_i);
+ *   dqk receives scale * dS x from both the query and the key side (keys are
+ *   the queries); dv_j += P_ij dout_i; a self-attending token passes dout
+ *   to dv. `out` and `lse` are lsh_attn_fwd's outputs for the same inputs.
+ */
+size_t lsh_bwd_workspace_size(const lsh_problem* p);
+lsh_status lsh_attn_bwd(const lsh_problem* p, const void* qk, const void* v,
+                        const int32_t* perm, const void* out, const float* lse,
+                        const void* dout, float* dqk, float* dv,
+                        void* ws, size_t ws_bytes, lsh_stream_t stream);
+
+/* Synchronises `stream`, returns and clears the current device's status
+ * word (LSH_OK, LSH_ERR_TIMEOUT or LSH_ERR_DEVICE_CHECK). */
+lsh_status lsh_device_status(lsh_stream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* lsh_status_string(lsh_status s);
+
+/* Number of kernels this library has launched in this process (a host-side
+ * counter, for accounting; never reset). */
+uint64_t lsh_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LSH_H */
