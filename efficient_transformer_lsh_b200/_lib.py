@@ -65,9 +65,9 @@ def lib() -> ctypes.CDLL:
             "lsh_sort_workspace_size": ([P], sz),
             "lsh_sort": ([P, vp, vp, vp, sz, vp], ctypes.c_int),
             "lsh_fwd_workspace_size": ([P], sz),
-            "lsh_attn_fwd": ([P, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+            "lsh_attn_fwd": ([P, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
             "lsh_bwd_workspace_size": ([P], sz),
-            "lsh_attn_bwd": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+            "lsh_attn_bwd": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
             "lsh_device_status": ([vp], ctypes.c_int),
             "lsh_status_string": ([ctypes.c_int], ctypes.c_char_p),
             "lsh_launch_count": ([], ctypes.c_uint64),
@@ -124,20 +124,21 @@ def lsh_fwd_workspace_size(p: lsh_problem) -> int:
     return int(lib().lsh_fwd_workspace_size(ctypes.byref(p)))
 
 
-def lsh_attn_fwd(p: lsh_problem, qk, v, perm, out, lse, ws, ws_bytes: int, stream=None):
-    _check(lib().lsh_attn_fwd(ctypes.byref(p), _ptr(qk), _ptr(v), _ptr(perm), _ptr(out), _ptr(lse),
-                              _ptr(ws), int(ws_bytes), _stream(stream)), "lsh_attn_fwd")
+def lsh_attn_fwd(p: lsh_problem, qk, v, perm, out, out_lo, lse, ws, ws_bytes: int, stream=None):
+    _check(lib().lsh_attn_fwd(ctypes.byref(p), _ptr(qk), _ptr(v), _ptr(perm), _ptr(out),
+                              _ptr(out_lo), _ptr(lse), _ptr(ws), int(ws_bytes), _stream(stream)),
+           "lsh_attn_fwd")
 
 
 def lsh_bwd_workspace_size(p: lsh_problem) -> int:
     return int(lib().lsh_bwd_workspace_size(ctypes.byref(p)))
 
 
-def lsh_attn_bwd(p: lsh_problem, qk, v, perm, out, lse, dout, dqk, dv, ws, ws_bytes: int,
+def lsh_attn_bwd(p: lsh_problem, qk, v, perm, out, out_lo, lse, dout, dqk, dv, ws, ws_bytes: int,
                  stream=None):
-    _check(lib().lsh_attn_bwd(ctypes.byref(p), _ptr(qk), _ptr(v), _ptr(perm), _ptr(out), _ptr(lse),
-                              _ptr(dout), _ptr(dqk), _ptr(dv), _ptr(ws), int(ws_bytes),
-                              _stream(stream)), "lsh_attn_bwd")
+    _check(lib().lsh_attn_bwd(ctypes.byref(p), _ptr(qk), _ptr(v), _ptr(perm), _ptr(out),
+                              _ptr(out_lo), _ptr(lse), _ptr(dout), _ptr(dqk), _ptr(dv), _ptr(ws),
+                              int(ws_bytes), _stream(stream)), "lsh_attn_bwd")
 
 
 def lsh_device_status(stream=None) -> int:

@@ -18,8 +18,8 @@ _TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
 class LSHAttention:
     """Reformer LSH self-attention for one fixed problem shape.
 
-    Buffers: bucket/perm [B,H,n_rounds,L] int32, out [B,H,L,d] (input dtype),
-    lse [B,H,L] float32, dqk/dv [B,H,L,d] float32, and the three workspaces.
+    Buffers: bucket/perm [B,H,n_rounds,L] int32, out and out_lo [B,H,L,d]
+    (input dtype; out_lo only for bf16), lse [B,H,L] float32, dqk/dv [B,H,L,d] float32, and the three workspaces.
     """
 
     def __init__(self, B, H, L, n_buckets, n_rounds, chunk, causal, dtype="bf16", d=64,
@@ -35,6 +35,9 @@ class LSHAttention:
         self.bucket = torch.empty((B, H, n_rounds, L), **i32)
         self.perm = torch.empty((B, H, n_rounds, L), **i32)
         self.out = torch.empty(self.shape, dtype=self.tdtype, device=dev)
+        # rounding residual of out (bf16 problems): keeps D = dout . O accurate
+        self.out_lo = torch.empty(self.shape, dtype=self.tdtype, device=dev) if dtype == "bf16" \
+            else None
         self.lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
         self.dqk = torch.empty(self.shape, dtype=torch.float32, device=dev)
         self.dv = torch.empty(self.shape, dtype=torch.float32, device=dev)
@@ -58,8 +61,8 @@ class LSHAttention:
         return self.perm
 
     def attend(self, qk, v, perm=None, stream=None):
-        _lib.lsh_attn_fwd(self.p, qk, v, self.perm if perm is None else perm, self.out, self.lse,
-                          self.ws_fwd, self.ws_fwd_bytes, stream)
+        _lib.lsh_attn_fwd(self.p, qk, v, self.perm if perm is None else perm, self.out,
+                          self.out_lo, self.lse, self.ws_fwd, self.ws_fwd_bytes, stream)
         return self.out, self.lse
 
     def forward(self, qk, v, R, stream=None):
@@ -70,8 +73,9 @@ class LSHAttention:
 
     def backward(self, qk, v, dout, perm=None, stream=None):
         """Gradients of sum(out * dout) w.r.t. qk and v (float32)."""
-        _lib.lsh_attn_bwd(self.p, qk, v, self.perm if perm is None else perm, self.out, self.lse,
-                          dout, self.dqk, self.dv, self.ws_bwd, self.ws_bwd_bytes, stream)
+        _lib.lsh_attn_bwd(self.p, qk, v, self.perm if perm is None else perm, self.out,
+                          self.out_lo, self.lse, dout, self.dqk, self.dv, self.ws_bwd,
+                          self.ws_bwd_bytes, stream)
         return self.dqk, self.dv
 
 

@@ -166,8 +166,8 @@ fwd_round_kernel(const T* __restrict__ qk, const T* __restrict__ v, const int32_
 template <typename T>
 __global__ void __launch_bounds__(256)
 combine_kernel(const float* __restrict__ opart, const float* __restrict__ lsepart,
-               const T* __restrict__ v, T* __restrict__ out, float* __restrict__ lse, int64_t N,
-               int n_rounds) {
+               const T* __restrict__ v, T* __restrict__ out, T* __restrict__ out_lo,
+               float* __restrict__ lse, int64_t N, int n_rounds) {
   const int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
   const int c4 = (threadIdx.x & 15) * 4;
   if (tok >= N) return;
@@ -175,6 +175,7 @@ combine_kernel(const float* __restrict__ opart, const float* __restrict__ lsepar
   for (int r = 0; r < n_rounds; ++r) mx = fmaxf(mx, lsepart[(int64_t)r * N + tok]);
   if (mx == -INFINITY) {
     store4(out + tok * kD + c4, load4(v + tok * kD + c4));
+    if (out_lo) store4(out_lo + tok * kD + c4, make_float4(0.f, 0.f, 0.f, 0.f));
     if (c4 == 0) lse[tok] = -INFINITY;
     return;
   }
@@ -190,19 +191,32 @@ combine_kernel(const float* __restrict__ opart, const float* __restrict__ lsepar
     acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
   }
   store4(out + tok * kD + c4, acc);
+  if (out_lo) {
+    float4 hi = load4(out + tok * kD + c4);   // the rounded value just stored
+    store4(out_lo + tok * kD + c4, make_float4(acc.x - hi.x, acc.y - hi.y, acc.z - hi.z,
+                                               acc.w - hi.w));
+  }
   if (c4 == 0) lse[tok] = LSE;
 }
 
 // D_i = dout_i . out_i; zero dqk; dv = dout for self-attending rows, else 0.
 template <typename T>
 __global__ void __launch_bounds__(256)
-bwd_prep_kernel(const T* __restrict__ out, const T* __restrict__ dout, const float* __restrict__ lse,
-                float* __restrict__ D, float* __restrict__ dqk, float* __restrict__ dv, int64_t N) {
+bwd_prep_kernel(const T* __restrict__ out, const T* __restrict__ out_lo, const T* __restrict__ dout,
+                const float* __restrict__ lse, float* __restrict__ D, float* __restrict__ dqk,
+                float* __restrict__ dv, int64_t N) {
   const int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
   const int c4 = (threadIdx.x & 15) * 4;
   const bool live = tok < N;
   float4 o = make_float4(0.f, 0.f, 0.f, 0.f), g = o;
-  if (live) { o = load4(out + tok * kD + c4); g = load4(dout + tok * kD + c4); }
+  if (live) {
+    o = load4(out + tok * kD + c4);
+    g = load4(dout + tok * kD + c4);
+    if (out_lo) {
+      float4 lo = load4(out_lo + tok * kD + c4);
+      o.x += lo.x; o.y += lo.y; o.z += lo.z; o.w += lo.w;
+    }
+  }
   float d = warp_sum16(o.x * g.x + o.y * g.y + o.z * g.z + o.w * g.w);
   if (!live) return;
   if (c4 == 0) D[tok] = d;
@@ -360,7 +374,7 @@ constexpr size_t kBwdSmem = (size_t)(4 * kQ + 2 * kK) * kP * 4 + (kQ + kK) * 4 +
 
 template <typename T>
 cudaError_t fwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* perm, T* out,
-                  float* lse, const FwdWs& ws, int* status, cudaStream_t s) {
+                  T* out_lo, float* lse, const FwdWs& ws, int* status, cudaStream_t s) {
   const int64_t N = (int64_t)p.B * p.H * p.L;
   const int64_t blocks = (int64_t)p.B * p.H * p.n_rounds * (p.L / kQ);
   cudaError_t e = cudaFuncSetAttribute(fwd_round_kernel<T>,
@@ -370,21 +384,22 @@ cudaError_t fwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* 
       qk, v, perm, ws.opart, ws.lsepart, p.L, p.chunk, p.n_rounds, N, p.causal,
       p.scale * kLog2e, status);
   combine_kernel<T><<<(unsigned)((N * 16 + 255) / 256), 256, 0, s>>>(ws.opart, ws.lsepart, v, out,
-                                                                     lse, N, p.n_rounds);
+                                                                     out_lo, lse, N, p.n_rounds);
   note_launch(2);
   return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t bwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* perm, const T* out,
-                  const float* lse, const T* dout, float* dqk, float* dv, float* D, int* status,
+                  const T* out_lo, const float* lse, const T* dout, float* dqk, float* dv, float* D, int* status,
                   cudaStream_t s) {
   const int64_t N = (int64_t)p.B * p.H * p.L;
   const int64_t blocks = (int64_t)p.B * p.H * p.n_rounds * (p.L / kQ);
   cudaError_t e = cudaFuncSetAttribute(bwd_round_kernel<T>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem);
   if (e != cudaSuccess) return e;
-  bwd_prep_kernel<T><<<(unsigned)((N * 16 + 255) / 256), 256, 0, s>>>(out, dout, lse, D, dqk, dv, N);
+  bwd_prep_kernel<T><<<(unsigned)((N * 16 + 255) / 256), 256, 0, s>>>(out, out_lo, dout, lse, D, dqk, dv,
+                                                                        N);
   bwd_round_kernel<T><<<(unsigned)blocks, 256, kBwdSmem, s>>>(
       qk, v, dout, perm, lse, D, dqk, dv, p.L, p.chunk, p.n_rounds, p.causal, p.scale,
       p.scale * kLog2e, status);
@@ -408,12 +423,13 @@ FwdWs fwd_ws_carve(const lsh_problem& p, void* ws) {
 }
 
 cudaError_t launch_attn_fwd(const lsh_problem& p, const void* qk, const void* v,
-                            const int32_t* perm, void* out, float* lse, const FwdWs& ws,
-                            int* status, cudaStream_t s) {
+                            const int32_t* perm, void* out, void* out_lo, float* lse,
+                            const FwdWs& ws, int* status, cudaStream_t s) {
   if (p.dtype == LSH_BF16)
     return fwd_t(p, (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, perm, (__nv_bfloat16*)out,
-                 lse, ws, status, s);
-  return fwd_t(p, (const float*)qk, (const float*)v, perm, (float*)out, lse, ws, status, s);
+                 (__nv_bfloat16*)out_lo, lse, ws, status, s);
+  return fwd_t(p, (const float*)qk, (const float*)v, perm, (float*)out, (float*)nullptr, lse, ws,
+               status, s);
 }
 
 size_t bwd_ws_bytes(const lsh_problem& p) {
@@ -421,15 +437,16 @@ size_t bwd_ws_bytes(const lsh_problem& p) {
 }
 
 cudaError_t launch_attn_bwd(const lsh_problem& p, const void* qk, const void* v,
-                            const int32_t* perm, const void* out, const float* lse,
-                            const void* dout, float* dqk, float* dv, void* ws, int* status,
-                            cudaStream_t s) {
+                            const int32_t* perm, const void* out, const void* out_lo,
+                            const float* lse, const void* dout, float* dqk, float* dv, void* ws,
+                            int* status, cudaStream_t s) {
   float* D = (float*)ws;
   if (p.dtype == LSH_BF16)
     return bwd_t(p, (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, perm,
-                 (const __nv_bfloat16*)out, lse, (const __nv_bfloat16*)dout, dqk, dv, D, status, s);
-  return bwd_t(p, (const float*)qk, (const float*)v, perm, (const float*)out, lse,
-               (const float*)dout, dqk, dv, D, status, s);
+                 (const __nv_bfloat16*)out, (const __nv_bfloat16*)out_lo, lse,
+                 (const __nv_bfloat16*)dout, dqk, dv, D, status, s);
+  return bwd_t(p, (const float*)qk, (const float*)v, perm, (const float*)out,
+               (const float*)nullptr, lse, (const float*)dout, dqk, dv, D, status, s);
 }
 
 }  // namespace lsh

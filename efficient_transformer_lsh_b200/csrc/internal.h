@@ -45,13 +45,13 @@ struct FwdWs {
 size_t fwd_ws_bytes(const lsh_problem& p);
 FwdWs fwd_ws_carve(const lsh_problem& p, void* ws);
 cudaError_t launch_attn_fwd(const lsh_problem& p, const void* qk, const void* v,
-                            const int32_t* perm, void* out, float* lse, const FwdWs& ws,
+                            const int32_t* perm, void* out, void* out_lo, float* lse, const FwdWs& ws,
                             int* status, cudaStream_t s);
 
 size_t bwd_ws_bytes(const lsh_problem& p);
 cudaError_t launch_attn_bwd(const lsh_problem& p, const void* qk, const void* v,
-                            const int32_t* perm, const void* out, const float* lse,
-                            const void* dout, float* dqk, float* dv, void* ws,
+                            const int32_t* perm, const void* out, const void* out_lo,
+                            const float* lse, const void* dout, float* dqk, float* dv, void* ws,
                             int* status, cudaStream_t s);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

@@ -105,14 +105,17 @@ size_t lsh_fwd_workspace_size(const lsh_problem* p) {
 }
 
 lsh_status lsh_attn_fwd(const lsh_problem* p, const void* qk, const void* v, const int32_t* perm,
-                        void* out, float* lse, void* ws, size_t ws_bytes, lsh_stream_t stream) {
+                        void* out, void* out_lo, float* lse, void* ws, size_t ws_bytes,
+                        lsh_stream_t stream) {
   lsh_status st = check_problem(p);
   if (st != LSH_OK) return st;
   if (empty(p)) return LSH_OK;
   if (!qk || !v || !perm || !out || !lse) return LSH_ERR_INVALID_ARG;
-  if (!aligned(qk, 16) || !aligned(v, 16) || !aligned(out, 16)) return LSH_ERR_INVALID_ARG;
+  if (!aligned(qk, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(out_lo, 16))
+    return LSH_ERR_INVALID_ARG;
   if (!ws || ws_bytes < fwd_ws_bytes(*p) || !aligned(ws, 256)) return LSH_ERR_WORKSPACE;
-  return cuda_status(launch_attn_fwd(*p, qk, v, perm, out, lse, fwd_ws_carve(*p, ws),
+  if (p->dtype == LSH_F32) out_lo = nullptr;
+  return cuda_status(launch_attn_fwd(*p, qk, v, perm, out, out_lo, lse, fwd_ws_carve(*p, ws),
                                      device_status_word(), (cudaStream_t)stream));
 }
 
@@ -122,17 +125,18 @@ size_t lsh_bwd_workspace_size(const lsh_problem* p) {
 }
 
 lsh_status lsh_attn_bwd(const lsh_problem* p, const void* qk, const void* v, const int32_t* perm,
-                        const void* out, const float* lse, const void* dout, float* dqk,
-                        float* dv, void* ws, size_t ws_bytes, lsh_stream_t stream) {
+                        const void* out, const void* out_lo, const float* lse, const void* dout,
+                        float* dqk, float* dv, void* ws, size_t ws_bytes, lsh_stream_t stream) {
   lsh_status st = check_problem(p);
   if (st != LSH_OK) return st;
   if (empty(p)) return LSH_OK;
   if (!qk || !v || !perm || !out || !lse || !dout || !dqk || !dv) return LSH_ERR_INVALID_ARG;
   if (!aligned(qk, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(dout, 16) ||
-      !aligned(dqk, 16) || !aligned(dv, 16))
+      !aligned(dqk, 16) || !aligned(dv, 16) || !aligned(out_lo, 16))
     return LSH_ERR_INVALID_ARG;
   if (!ws || ws_bytes < bwd_ws_bytes(*p) || !aligned(ws, 256)) return LSH_ERR_WORKSPACE;
-  return cuda_status(launch_attn_bwd(*p, qk, v, perm, out, lse, dout, dqk, dv, ws,
+  if (p->dtype == LSH_F32) out_lo = nullptr;
+  return cuda_status(launch_attn_bwd(*p, qk, v, perm, out, out_lo, lse, dout, dqk, dv, ws,
                                      device_status_word(), (cudaStream_t)stream));
 }
 

@@ -30,7 +30,7 @@
  *   - Outputs are overwritten, never accumulated into.
  *   - Shapes: B batch, H heads, L sequence length, d head size (64),
  *     n_buckets (even), n_rounds hash rounds, chunk = m.
- *     qk, v, out, dout: [B, H, L, d] in `dtype`;
+ *     qk, v, out, out_lo, dout: [B, H, L, d] in `dtype`;
  *     R: [n_rounds, d, n_buckets/2] in `dtype`;
  *     bucket, perm: [B, H, n_rounds, L] int32;
  *     lse: [B, H, L] float32; dqk, dv: [B, H, L, d] float32.
@@ -101,10 +101,14 @@ lsh_status lsh_sort(const lsh_problem* p, const int32_t* bucket, int32_t* perm,
  *   lse[i] = log sum_r exp(lse_r,i), out[i] = sum_r exp(lse_r,i - lse[i]) o_r,i.
  *   A token with no valid key in any round attends to itself:
  *   out[i] = v[i], lse[i] = -inf.
+ *   out_lo (optional, may be NULL; same shape and dtype as out): for bf16
+ *   problems, the rounding residual out_lo = bf16(O - out) of the float32
+ *   result O, so that out + out_lo carries O to about 16 significant bits;
+ *   lsh_attn_bwd uses it for D = dout . O. Ignored for float32 problems.
  */
 size_t lsh_fwd_workspace_size(const lsh_problem* p);
 lsh_status lsh_attn_fwd(const lsh_problem* p, const void* qk, const void* v,
-                        const int32_t* perm, void* out, float* lse,
+                        const int32_t* perm, void* out, void* out_lo, float* lse,
                         void* ws, size_t ws_bytes, lsh_stream_t stream);
 
 /*
@@ -114,12 +118,14 @@ lsh_status lsh_attn_fwd(const lsh_problem* p, const void* qk, const void* v,
  *   Summary paragraph). D_i = dout_i . out_i; dS = P (dout_i . v_j - D_i);
  *   dqk receives scale * dS x from both the query and the key side (keys are
  *   the queries); dv_j += P_ij dout_i; a self-attending token passes dout
- *   to dv. `out` and `lse` are lsh_attn_fwd's outputs for the same inputs.
+ *   to dv. `out`, `out_lo` and `lse` are lsh_attn_fwd's outputs for the same
+ *   inputs; out_lo may be NULL, in which case D is formed from `out` alone
+ *   (for bf16 problems that adds the rounding error of out to D).
  */
 size_t lsh_bwd_workspace_size(const lsh_problem* p);
 lsh_status lsh_attn_bwd(const lsh_problem* p, const void* qk, const void* v,
-                        const int32_t* perm, const void* out, const float* lse,
-                        const void* dout, float* dqk, float* dv,
+                        const int32_t* perm, const void* out, const void* out_lo,
+                        const float* lse, const void* dout, float* dqk, float* dv,
                         void* ws, size_t ws_bytes, lsh_stream_t stream);
 
 /* Synchronises `stream`, returns and clears the current device's status

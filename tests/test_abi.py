@@ -63,7 +63,8 @@ def test_bad_problem_rejected_before_launch(kw, code):
     r = L.lsh_hash(ctypes.byref(p), FAKE, FAKE, FAKE, None)
     assert r == code
     assert L.lsh_sort_workspace_size(ctypes.byref(p)) == 0
-    assert L.lsh_attn_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == code
+    assert L.lsh_attn_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30,
+                          None) == code
 
 
 def test_null_pointers_and_workspace_rejected():
@@ -80,12 +81,15 @@ def test_null_pointers_and_workspace_rejected():
     assert L.lsh_sort(ctypes.byref(p), FAKE, FAKE, FAKE + 16, need, None) == 3
     assert L.lsh_sort(ctypes.byref(p), None, FAKE, FAKE, need, None) == 1
     nf = L.lsh_fwd_workspace_size(ctypes.byref(p))
-    assert L.lsh_attn_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, nf - 1, None) == 3
+    assert L.lsh_attn_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, nf - 1,
+                          None) == 3
+    assert L.lsh_attn_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE + 8, FAKE, FAKE, nf,
+                          None) == 1   # misaligned out_lo
     nb = L.lsh_bwd_workspace_size(ctypes.byref(p))
-    assert L.lsh_attn_bwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
-                          nb - 1, None) == 3
-    assert L.lsh_attn_bwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE,
-                          nb, None) == 1
+    assert L.lsh_attn_bwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE,
+                          FAKE, nb - 1, None) == 3
+    assert L.lsh_attn_bwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, FAKE,
+                          FAKE, nb, None) == 1
 
 
 def test_empty_problem_is_a_noop():
@@ -95,9 +99,10 @@ def test_empty_problem_is_a_noop():
         p = _p(**kw)
         assert L.lsh_hash(ctypes.byref(p), None, None, None, None) == 0
         assert L.lsh_sort(ctypes.byref(p), None, None, None, 0, None) == 0
-        assert L.lsh_attn_fwd(ctypes.byref(p), None, None, None, None, None, None, 0, None) == 0
+        assert L.lsh_attn_fwd(ctypes.byref(p), None, None, None, None, None, None, None, 0,
+                              None) == 0
         assert L.lsh_attn_bwd(ctypes.byref(p), None, None, None, None, None, None, None, None,
-                              None, 0, None) == 0
+                              None, None, 0, None) == 0
 
 
 def test_workspace_sizes_grow_with_problem():

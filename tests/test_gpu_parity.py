@@ -53,7 +53,8 @@ def test_identical_tokens_all_in_one_bucket():
     inp = generate(w)
     inp["qk"][:] = inp["qk"][:, :, :1, :]
     ref = oracle_run(w, inp, True)
-    assert np.all(ref["bucket"] == ref["bucket"].flat[0])
+    for r in range(w.n_rounds):     # one bucket per round
+        assert np.all(ref["bucket"][:, :, r] == ref["bucket"][0, 0, r, 0])
     got = gpu_run(w, inp, ref["bucket"], True)
     compare(w, ref, got, True, label="identical")
 
@@ -90,7 +91,8 @@ def test_launch_counter_moves():
 def test_autograd_wrapper_matches_oracle():
     import torch
     from efficient_transformer_lsh_b200.attention import lsh_attention
-    w = CASES["batch-small"]
+    # one chunk spanning the sequence: the result does not depend on bucket ids
+    w = CASES["bf16-one-chunk"]
     inp = generate(w)
     ref = oracle_run(w, inp, True)
     dev = torch.device("cuda")
@@ -99,9 +101,7 @@ def test_autograd_wrapper_matches_oracle():
     R = torch.from_numpy(inp["R"]).to(dev).to(torch.bfloat16)
     out, lse = lsh_attention(qk, v, R, w.n_buckets, w.chunk, w.causal, w.scale)
     (out.float() * torch.from_numpy(inp["dO"]).to(dev)).sum().backward()
-    near = (ref["gap"] < 1e-5).any()
-    if not near:
-        assert np.abs(out.float().cpu().numpy() - ref["O"]).max() <= 2e-2
-        # bf16 gradients: the tolerance includes one bf16 rounding of the result
-        assert np.abs(qk.grad.float().cpu().numpy() - ref["dqk"]).max() <= 4e-2
-        assert np.abs(v.grad.float().cpu().numpy() - ref["dv"]).max() <= 4e-2
+    assert np.abs(out.detach().float().cpu().numpy() - ref["O"]).max() <= 2e-2
+    # bf16 gradients: the tolerance includes one bf16 rounding of the result
+    assert np.abs(qk.grad.float().cpu().numpy() - ref["dqk"]).max() <= 4e-2
+    assert np.abs(v.grad.float().cpu().numpy() - ref["dv"]).max() <= 4e-2
