@@ -21,7 +21,9 @@ STATUS_NAMES = {
 # Every symbol include/lsh.h declares.
 EXPORTS = ("lsh_hash", "lsh_sort_workspace_size", "lsh_sort", "lsh_fwd_workspace_size",
            "lsh_attn_fwd", "lsh_bwd_workspace_size", "lsh_attn_bwd", "lsh_device_status",
-           "lsh_status_string", "lsh_launch_count")
+           "lsh_status_string", "lsh_launch_count", "lsh_sort_noalloc")
+# Size of the library-owned scratch used by lsh_sort_noalloc (matches lsh.h).
+SORT_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class LshLibraryMissing(RuntimeError):
@@ -71,6 +73,7 @@ def lib() -> ctypes.CDLL:
             "lsh_device_status": ([vp], ctypes.c_int),
             "lsh_status_string": ([ctypes.c_int], ctypes.c_char_p),
             "lsh_launch_count": ([], ctypes.c_uint64),
+            "lsh_sort_noalloc": ([P, vp, vp, vp], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -118,6 +121,12 @@ def lsh_sort_workspace_size(p: lsh_problem) -> int:
 def lsh_sort(p: lsh_problem, bucket, perm, ws, ws_bytes: int, stream=None):
     _check(lib().lsh_sort(ctypes.byref(p), _ptr(bucket), _ptr(perm), _ptr(ws), int(ws_bytes),
                           _stream(stream)), "lsh_sort")
+
+
+def lsh_sort_noalloc(p: lsh_problem, bucket, perm, stream=None):
+    """lsh_sort for callers that cannot provide a workspace (library-owned scratch)."""
+    _check(lib().lsh_sort_noalloc(ctypes.byref(p), _ptr(bucket), _ptr(perm), _stream(stream)),
+           "lsh_sort_noalloc")
 
 
 def lsh_fwd_workspace_size(p: lsh_problem) -> int:

@@ -216,3 +216,56 @@ cudaError_t launch_sort(const lsh_problem& p, const int32_t* bucket, int32_t* pe
 }
 
 }  // namespace lsh
+
+// ----------------------------------------------------------------------------
+// Sort with library-owned scratch, for callers that cannot hand the library a
+// workspace (see lsh_sort_noalloc in lsh.h).
+// ----------------------------------------------------------------------------
+#include <mutex>
+
+namespace lsh {
+namespace {
+
+// Shared scratch for every lsh_sort_noalloc call on a device. Each GPU that
+// loads the library holds these bytes until the process exits.
+static __device__ __align__(256) unsigned char g_sort_scratch[LSH_SORT_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kScratchDevices = 64;
+void* g_sort_scratch_addr[kScratchDevices] = {};
+std::mutex g_sort_scratch_mu;
+
+// Device address of g_sort_scratch on the current device. The host-side name
+// of the array is only a stand-in, so the address is looked up once per
+// device with that device current, and cached.
+cudaError_t sort_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kScratchDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_sort_scratch_mu);
+  if (!g_sort_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_sort_scratch);
+    if (e != cudaSuccess) return e;
+    g_sort_scratch_addr[dev] = ptr;
+  }
+  *out = g_sort_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace lsh
+
+extern "C" lsh_status lsh_sort_noalloc(const lsh_problem* p, const int32_t* bucket, int32_t* perm,
+                                       lsh_stream_t stream) {
+  // Invalid and empty problems report a zero workspace size; lsh_sort then
+  // returns their status without touching the device.
+  const size_t need = lsh_sort_workspace_size(p);
+  if (need == 0) return lsh_sort(p, bucket, perm, nullptr, 0, stream);
+  if (need > (size_t)LSH_SORT_NOALLOC_SCRATCH_BYTES) return LSH_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (lsh::sort_scratch_address(&scratch) != cudaSuccess) return LSH_ERR_CUDA;
+  // lsh_sort clears the per-tile counters it needs on the stream before use;
+  // everything else in the scratch is overwritten.
+  return lsh_sort(p, bucket, perm, scratch, (size_t)LSH_SORT_NOALLOC_SCRATCH_BYTES, stream);
+}

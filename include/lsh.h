@@ -128,6 +128,32 @@ lsh_status lsh_attn_bwd(const lsh_problem* p, const void* qk, const void* v,
                         const float* lse, const void* dout, float* dqk, float* dv,
                         void* ws, size_t ws_bytes, lsh_stream_t stream);
 
+/*
+ * lsh_sort_noalloc — lsh_sort without a caller workspace. The reference pages
+ *   have no counterpart: this entry point exists for callers that cannot
+ *   obtain device memory for a workspace, such as a host framework that owns
+ *   every byte of device memory and gives kernel libraries no allocation hook,
+ *   or a latency-critical loop where cudaMalloc's implicit device-wide
+ *   synchronisation is not acceptable. It allocates nothing: its scratch is
+ *   one array of LSH_SORT_NOALLOC_SCRATCH_BYTES (16 MiB) in the library's own
+ *   device memory, which every GPU that loads the library holds until the
+ *   process exits.
+ *   - Same arguments, result and checks as lsh_sort. A problem whose
+ *     lsh_sort_workspace_size() exceeds the scratch returns LSH_ERR_WORKSPACE
+ *     and launches nothing. (16 MiB covers, e.g., 8 heads x 4 rounds x 65536
+ *     positions with 1024 buckets, or 2 x 524288 positions with 8192.)
+ *   - All calls on a device share the one scratch array and it keeps the last
+ *     call's contents; the sort clears what must start at zero itself. Calls
+ *     whose work overlaps on the GPU (other streams, other host threads)
+ *     race on the scratch and give wrong results: serialise them.
+ *   - The first call on each device looks up the scratch's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ */
+#define LSH_SORT_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+lsh_status lsh_sort_noalloc(const lsh_problem* p, const int32_t* bucket, int32_t* perm,
+                            lsh_stream_t stream);
+
 /* Synchronises `stream`, returns and clears the current device's status
  * word (LSH_OK, LSH_ERR_TIMEOUT or LSH_ERR_DEVICE_CHECK). */
 lsh_status lsh_device_status(lsh_stream_t stream);
