@@ -163,9 +163,11 @@ fwd_round_kernel(const T* __restrict__ qk, const T* __restrict__ v, const int32_
 }
 
 // Round combine in original order; 16 threads per token, 4 columns each.
-template <typename T>
+// PT: type of the per-round outputs (float from the CUDA-core kernel, __half
+// from the tensor-core kernel).
+template <typename T, typename PT>
 __global__ void __launch_bounds__(256)
-combine_kernel(const float* __restrict__ opart, const float* __restrict__ lsepart,
+combine_kernel(const PT* __restrict__ opart, const float* __restrict__ lsepart,
                const T* __restrict__ v, T* __restrict__ out, T* __restrict__ out_lo,
                float* __restrict__ lse, int64_t N, int n_rounds) {
   const int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
@@ -377,14 +379,23 @@ cudaError_t fwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* 
                   T* out_lo, float* lse, const FwdWs& ws, int* status, cudaStream_t s) {
   const int64_t N = (int64_t)p.B * p.H * p.L;
   const int64_t blocks = (int64_t)p.B * p.H * p.n_rounds * (p.L / kQ);
-  cudaError_t e = cudaFuncSetAttribute(fwd_round_kernel<T>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFwdSmem);
+  const unsigned cblocks = (unsigned)((N * 16 + 255) / 256);
+  cudaError_t e = launch_attn_fwd_tc(p, qk, v, perm, ws.opart, ws.lsepart, status, s);
+  if (e == cudaSuccess) {
+    combine_kernel<T, __half><<<cblocks, 256, 0, s>>>((const __half*)ws.opart, ws.lsepart, v, out,
+                                                      out_lo, lse, N, p.n_rounds);
+    note_launch();
+    return cudaGetLastError();
+  }
+  if (e != cudaErrorNotSupported) return e;
+  e = cudaFuncSetAttribute(fwd_round_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kFwdSmem);
   if (e != cudaSuccess) return e;
   fwd_round_kernel<T><<<(unsigned)blocks, 256, kFwdSmem, s>>>(
       qk, v, perm, ws.opart, ws.lsepart, p.L, p.chunk, p.n_rounds, N, p.causal,
       p.scale * kLog2e, status);
-  combine_kernel<T><<<(unsigned)((N * 16 + 255) / 256), 256, 0, s>>>(ws.opart, ws.lsepart, v, out,
-                                                                     out_lo, lse, N, p.n_rounds);
+  combine_kernel<T, float><<<cblocks, 256, 0, s>>>(ws.opart, ws.lsepart, v, out, out_lo, lse, N,
+                                                   p.n_rounds);
   note_launch(2);
   return cudaGetLastError();
 }

@@ -48,6 +48,12 @@ cudaError_t launch_attn_fwd(const lsh_problem& p, const void* qk, const void* v,
                             const int32_t* perm, void* out, void* out_lo, float* lse, const FwdWs& ws,
                             int* status, cudaStream_t s);
 
+// tcgen05 per-round forward (bf16, chunk 64): writes fp16 per-round outputs
+// [n_rounds][B*H*L][64] and lse_r; cudaErrorNotSupported for other shapes.
+cudaError_t launch_attn_fwd_tc(const lsh_problem& p, const void* qk, const void* v,
+                               const int32_t* perm, void* opart_f16, float* lsepart, int* status,
+                               cudaStream_t s);
+
 size_t bwd_ws_bytes(const lsh_problem& p);
 cudaError_t launch_attn_bwd(const lsh_problem& p, const void* qk, const void* v,
                             const int32_t* perm, const void* out, const void* out_lo,
