@@ -14,20 +14,26 @@
 //
 // Warp roles (persistent CTA, one per SM, walking units of kUnit pairs of one
 // (batch, head, round) segment):
-//   warps 0-3 : gather rows of x and v through perm (16-byte loads), convert
-//               bf16 -> fp16 (exact for |values| < 65504), store them in the
-//               128-byte-swizzled K-major layout into a 4-slot ring; chunk
-//               2p0-1 of a unit's first pair goes to a separate buffer;
-//   warp 4    : TMEM allocation; one thread issues S = Q K^T (3 MMAs of
-//               128x64x64 per pair into a double-buffered TMEM S) and
-//               O = P V (P from shared memory, V as the MN-major operand);
-//   warps 5-8 : softmax, one query row per thread: S from TMEM, masks
-//               (causal / self), row max, exp2, row sum, P (fp16) into shared
-//               memory; then O from TMEM, scaled by 1/l, written as the fp16
-//               per-round output in original token order with lse_r.
-// fp16 operands for P V keep P's rounding error at 2^-11 (bf16 would add
-// about 3e-3 to O on the 64K workload).
+//   warps 0-3  : producers — cp.async gathers of x and v rows through perm
+//                straight into the 128-byte-swizzled K-major layout of a
+//                4-slot ring (a unit's first pair also needs chunk 2p0-1,
+//                which goes to one of 3 rotating side buffers); each thread
+//                then converts its own pieces bf16 -> fp16 in place (exact
+//                for |values| < 65504). Software-pipelined one job deep;
+//   warp 4     : TMEM allocation; one thread issues S = Q K^T (three
+//                128x64x64 MMAs per pair into a double-buffered TMEM S) and
+//                O = P V with P read from TMEM (A operand) and V from shared
+//                memory (MN-major B operand);
+//   warps 5-8  : softmax warpgroup for even jobs, warps 9-12 for odd jobs —
+//                one query row per thread, two passes over its S row in TMEM:
+//                (1) causal/self mask and row max, masked values written back;
+//                (2) exp2, row sum, P packed as fp16 pairs into TMEM over S.
+//                The warpgroup then writes its previous job's output: O from
+//                TMEM scaled by 1/l, as fp16, in original token order, + lse_r.
+// fp16 for P and V keeps P's rounding error at 2^-11 (bf16 would add about
+// 3e-3 to O on the 64K workload).
 #include <cuda_fp16.h>
+#include <stddef.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -42,35 +48,39 @@ using namespace tc;
 constexpr int kM = 64;            // chunk
 constexpr int kUnit = 8;          // pairs per work unit
 constexpr int kSlots = 4;         // pair slots in the ring
-constexpr int kTile = 64 * 128;   // one chunk of 64 rows x 64 fp16 = 8 KB
+constexpr int kPre = 3;           // side buffers for a unit's previous chunk
+constexpr int kTile = 64 * 128;   // one chunk of 64 rows x 64 16-bit values = 8 KB
 constexpr int kSlotBytes = 4 * kTile;   // x_even | x_odd | v_even | v_odd
 constexpr int kPreBytes = 2 * kTile;    // x_prev | v_prev
-constexpr int kPBytes = 3 * 128 * 128;  // P: 3 blocks of 128 rows x 64 fp16
-constexpr int kThreads = 288;
-constexpr uint32_t kSCols = 192;
+constexpr int kThreads = 416;
+constexpr uint32_t kSCols = 192;        // TMEM columns of one S / P buffer
+constexpr uint32_t kOCol = 2 * kSCols;  // first TMEM column of the O buffers
 
-struct __align__(8) FwdBar {
+struct __align__(16) FwdBar {
   uint64_t slot_full[kSlots];
   uint64_t slot_free[kSlots];
-  uint64_t pre_free;
+  uint64_t pre_free[kPre];
   uint64_t s_full[2];
-  uint64_t s_free[2];
-  uint64_t p_full;
-  uint64_t p_free;
+  uint64_t p_full[2];
+  uint64_t p_free[2];
   uint64_t o_free[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
-  int kpos[kSlots][128];   // original positions of the slot's even|odd rows
-  int kpos_pre[64];
+  // original positions of the slot's even|odd rows; read as int4, so
+  // 16-byte aligned
+  alignas(16) int kpos[kSlots][128];
+  alignas(16) int kpos_pre[kPre][64];
 };
+static_assert(offsetof(FwdBar, kpos) % 16 == 0 && offsetof(FwdBar, kpos_pre) % 16 == 0,
+              "position arrays are read with 16-byte loads");
 
-constexpr size_t kSmemBytes = 1024 + kSlots * kSlotBytes + kPreBytes + kPBytes + sizeof(FwdBar);
+constexpr size_t kSmemBytes = 1024 + kSlots * kSlotBytes + kPre * kPreBytes + sizeof(FwdBar);
 
 struct Job {
   int64_t seg;   // (b*H + h)*n_rounds + r
   int p;         // pair index within the segment
-  bool first;    // first pair of its unit (its previous chunk is gathered separately)
+  bool first;    // first pair of its unit
 };
 
 // Walks the CTA's units in order; every role iterates the same sequence.
@@ -82,8 +92,7 @@ struct JobIter {
   __device__ bool next(Job& j) {
     while (unit < n_units) {
       const int64_t seg = unit / units_per_seg;
-      const int p0 = (int)(unit % units_per_seg) * kUnit;
-      const int p = p0 + k;
+      const int p = (int)(unit % units_per_seg) * kUnit + k;
       if (k < kUnit && p < n_pairs) {
         j.seg = seg;
         j.p = p;
@@ -104,60 +113,54 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-
-__device__ __forceinline__ uint32_t cvt_bf16x2_to_f16x2(uint32_t u) {
-  const float lo = __uint_as_float(u << 16), hi = __uint_as_float(u & 0xffff0000u);
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
-// Gathers the 64 rows of chunk c of segment `seg` (x and v), converting to fp16
-// and storing swizzled. Thread t: row t>>1, 16-byte chunks 4*(t&1)..+3.
-__device__ __forceinline__ void gather_chunk(const __nv_bfloat16* __restrict__ qk,
-                                             const __nv_bfloat16* __restrict__ v,
-                                             const int32_t* __restrict__ perm, int64_t seg,
-                                             int64_t bh, int L, int c, uint8_t* x_dst,
-                                             uint8_t* v_dst, int* kpos, int t, int* status) {
-  const int row = t >> 1, half = t & 1;
+// Position of row `row` of chunk c, checked against L (a bad id is recorded
+// in the status word and replaced by 0 so no copy leaves the tensor).
+__device__ __forceinline__ int chunk_pos(const int32_t* __restrict__ perm, int64_t seg, int L, int c,
+                                         int row, int* status) {
   int pos = perm[seg * L + (int64_t)c * kM + row];
   if ((unsigned)pos >= (unsigned)L) {
     if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
     pos = 0;
   }
-  if (half == 0) kpos[row] = pos;
-  const uint4* xs = reinterpret_cast<const uint4*>(qk + (bh * L + pos) * 64) + half * 4;
-  const uint4* vs = reinterpret_cast<const uint4*>(v + (bh * L + pos) * 64) + half * 4;
-  uint4 xv[4], vv[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    xv[i] = __ldg(xs + i);
-    vv[i] = __ldg(vs + i);
-  }
+  return pos;
+}
+
+// Thread t copies 16-byte pieces 4*(t&1)..+3 of row t>>1 of a chunk tile into
+// their 128-byte-swizzled places (bf16; converted later in place).
+__device__ __forceinline__ void issue_row(const __nv_bfloat16* __restrict__ src_row, uint8_t* tile,
+                                          int row, int half) {
+  const uint32_t base = smem_u32(tile) + row * 128;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int ch = half * 4 + i;
-    const uint32_t off = row * 128 + ((ch ^ (row & 7)) << 4);
-    uint4 a, b;
-    a.x = cvt_bf16x2_to_f16x2(xv[i].x); a.y = cvt_bf16x2_to_f16x2(xv[i].y);
-    a.z = cvt_bf16x2_to_f16x2(xv[i].z); a.w = cvt_bf16x2_to_f16x2(xv[i].w);
-    b.x = cvt_bf16x2_to_f16x2(vv[i].x); b.y = cvt_bf16x2_to_f16x2(vv[i].y);
-    b.z = cvt_bf16x2_to_f16x2(vv[i].z); b.w = cvt_bf16x2_to_f16x2(vv[i].w);
-    *reinterpret_cast<uint4*>(x_dst + off) = a;
-    *reinterpret_cast<uint4*>(v_dst + off) = b;
+    cp_async16(base + (((uint32_t)ch ^ (uint32_t)(row & 7)) << 4), src_row + ch * 8);
+  }
+}
+__device__ __forceinline__ void convert_row(uint8_t* tile, int row, int half) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int ch = half * 4 + i;
+    convert_piece_bf16_to_f16(tile + row * 128 + ((ch ^ (row & 7)) << 4));
   }
 }
 
+template <bool kCausal>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __restrict__ v,
                    const int32_t* __restrict__ perm, __half* __restrict__ opart,
-                   float* __restrict__ lsepart, int L, int n_rounds, int64_t N, int causal,
-                   float scale_log2, int64_t n_units, int units_per_seg, int* status) {
+                   float* __restrict__ lsepart, int L, int n_rounds, int64_t N, float scale_log2,
+                   int64_t n_units, int units_per_seg, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* slots = smem;
-  uint8_t* pre = slots + kSlots * kSlotBytes;
-  uint8_t* pbuf = pre + kPreBytes;
-  FwdBar* bar = (FwdBar*)(pbuf + kPBytes);
+  uint8_t* pres = slots + kSlots * kSlotBytes;
+  FwdBar* bar = (FwdBar*)(pres + kPre * kPreBytes);
   volatile int* abort = &bar->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -169,14 +172,13 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
       mbar_init(&bar->slot_full[s], 128);
       mbar_init(&bar->slot_free[s], 1);
     }
-    mbar_init(&bar->pre_free, 1);
+    for (int s = 0; s < kPre; ++s) mbar_init(&bar->pre_free[s], 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar->s_full[b], 1);
-      mbar_init(&bar->s_free[b], 128);
+      mbar_init(&bar->p_full[b], 128);
+      mbar_init(&bar->p_free[b], 1);
       mbar_init(&bar->o_free[b], 128);
     }
-    mbar_init(&bar->p_full, 128);
-    mbar_init(&bar->p_free, 1);
     mbar_init(&bar->mma_done, 1);
     bar->abort = 0;
     fence_mbar_init();
@@ -192,101 +194,166 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
 
   if (warp < 4) {
     // ------------------------------------------------ producers
-    const int t = threadIdx.x;
+    const int t = threadIdx.x, row = t >> 1, half = t & 1;
     JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
-    Job j;
+    Job cur, nxt;
+    bool have_cur = it.next(cur);
+    int pos_p = 0, pos_e = 0, pos_o = 0;
+    auto fetch_pos = [&](const Job& jb) {
+      pos_e = chunk_pos(perm, jb.seg, L, 2 * jb.p, row, status);
+      pos_o = (2 * jb.p + 1 < n_chunks) ? chunk_pos(perm, jb.seg, L, 2 * jb.p + 1, row, status) : 0;
+      pos_p = (jb.first && jb.p > 0) ? chunk_pos(perm, jb.seg, L, 2 * jb.p - 1, row, status) : 0;
+    };
+    if (have_cur) fetch_pos(cur);
     int n = 0, pre_uses = 0;
-    while (it.next(j)) {
+    bool pend = false, pend_odd = false;
+    int pend_slot = 0, pend_pre = -1;
+    bool ok = true;
+    auto publish = [&]() {
+      uint8_t* ps = slots + pend_slot * kSlotBytes;
+      if (pend_pre >= 0) {
+        uint8_t* pb = pres + pend_pre * kPreBytes;
+        convert_row(pb, row, half);
+        convert_row(pb + kTile, row, half);
+      }
+      convert_row(ps, row, half);
+      convert_row(ps + 2 * kTile, row, half);
+      if (pend_odd) {
+        convert_row(ps + kTile, row, half);
+        convert_row(ps + 3 * kTile, row, half);
+      }
+      fence_proxy_async();
+      mbar_arrive(&bar->slot_full[pend_slot]);
+    };
+    while (have_cur) {
       const int s = n % kSlots;
       if (n >= kSlots &&
-          !mbar_wait(&bar->slot_free[s], (uint32_t)(n / kSlots - 1) & 1u, abort, status))
+          !mbar_wait(&bar->slot_free[s], (uint32_t)(n / kSlots - 1) & 1u, abort, status)) {
+        ok = false;
         break;
-      const int64_t bh = j.seg / n_rounds;
-      uint8_t* sl = slots + s * kSlotBytes;
-      const int ce = 2 * j.p, co = 2 * j.p + 1;
-      if (j.first && j.p > 0) {
-        if (pre_uses > 0 &&
-            !mbar_wait(&bar->pre_free, (uint32_t)(pre_uses - 1) & 1u, abort, status))
+      }
+      const bool use_pre = cur.first && cur.p > 0, has_odd = 2 * cur.p + 1 < n_chunks;
+      int pb_idx = -1;
+      if (use_pre) {
+        pb_idx = pre_uses % kPre;
+        if (pre_uses >= kPre &&
+            !mbar_wait(&bar->pre_free[pb_idx], (uint32_t)(pre_uses / kPre - 1) & 1u, abort,
+                       status)) {
+          ok = false;
           break;
-        gather_chunk(qk, v, perm, j.seg, bh, L, ce - 1, pre, pre + kTile, bar->kpos_pre, t, status);
+        }
         ++pre_uses;
       }
-      gather_chunk(qk, v, perm, j.seg, bh, L, ce, sl, sl + 2 * kTile, bar->kpos[s], t, status);
-      if (co < n_chunks)
-        gather_chunk(qk, v, perm, j.seg, bh, L, co, sl + kTile, sl + 3 * kTile, bar->kpos[s] + 64,
-                     t, status);
-      fence_proxy_async();
-      mbar_arrive(&bar->slot_full[s]);
+      const int64_t bh = cur.seg / n_rounds;
+      uint8_t* sl = slots + s * kSlotBytes;
+      const __nv_bfloat16* xb = qk + bh * L * 64;
+      const __nv_bfloat16* vb = v + bh * L * 64;
+      if (use_pre) {
+        uint8_t* pb = pres + pb_idx * kPreBytes;
+        if (half == 0) bar->kpos_pre[pb_idx][row] = pos_p;
+        issue_row(xb + (int64_t)pos_p * 64, pb, row, half);
+        issue_row(vb + (int64_t)pos_p * 64, pb + kTile, row, half);
+      }
+      if (half == 0) bar->kpos[s][row] = pos_e;
+      issue_row(xb + (int64_t)pos_e * 64, sl, row, half);
+      issue_row(vb + (int64_t)pos_e * 64, sl + 2 * kTile, row, half);
+      if (has_odd) {
+        if (half == 0) bar->kpos[s][64 + row] = pos_o;
+        issue_row(xb + (int64_t)pos_o * 64, sl + kTile, row, half);
+        issue_row(vb + (int64_t)pos_o * 64, sl + 3 * kTile, row, half);
+      }
+      cp_async_commit();
+      have_cur = it.next(nxt);
+      if (have_cur) fetch_pos(nxt);
+      if (pend) {
+        cp_async_wait<1>();
+        publish();
+      }
+      pend = true;
+      pend_slot = s;
+      pend_pre = pb_idx;
+      pend_odd = has_odd;
+      cur = nxt;
       ++n;
     }
+    cp_async_wait<0>();
+    if (pend && ok) publish();
   } else if (warp == 4) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = idesc_f16(128, 64, 0, false, false);   // Q K^T, both K-major
       const uint32_t idesc_o = idesc_f16(128, 64, 0, false, true);    // P V, V MN-major
-      const uint32_t slots_a = smem_u32(slots), pre_a = smem_u32(pre), p_a = smem_u32(pbuf);
+      const uint32_t slots_a = smem_u32(slots), pres_a = smem_u32(pres);
       JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
       Job cur, nxt;
       bool have_cur = it.next(cur);
-      int n = 0;
+      int n = 0, pre_uses = 0;
+      int cur_pre = -1, nxt_pre = -1;
       bool ok = true;
-      // issue S for job n (slot n%kSlots, buffer n&1)
-      auto issue_s = [&](const Job& jb, int nn) -> bool {
+      // S for job nn (slot nn % kSlots, TMEM buffer nn & 1)
+      auto issue_s = [&](const Job& jb, int nn, int pb) -> bool {
         const int s = nn % kSlots, b = nn & 1;
         if (!mbar_wait(&bar->slot_full[s], (uint32_t)(nn / kSlots) & 1u, abort, status)) return false;
-        if (nn >= 2 && !mbar_wait(&bar->s_free[b], (uint32_t)(nn / 2 - 1) & 1u, abort, status))
-          return false;
         tc_fence_after();
         const uint32_t sl = slots_a + s * kSlotBytes;
         const uint32_t d = tmem + (uint32_t)b * kSCols;
         const bool has_prev = jb.p > 0, has_odd = 2 * jb.p + 1 < n_chunks;
-        const uint32_t prev_x =
-            jb.first ? pre_a : slots_a + ((nn + kSlots - 1) % kSlots) * kSlotBytes + kTile;
-        const uint32_t keys[3] = {prev_x, sl, sl + kTile};
+        const uint32_t prev_x = pb >= 0 ? pres_a + pb * kPreBytes
+                                        : slots_a + ((nn + kSlots - 1) % kSlots) * kSlotBytes + kTile;
+#pragma unroll
         for (int kb = 0; kb < 3; ++kb) {
           if ((kb == 0 && !has_prev) || (kb == 2 && !has_odd)) continue;
+          const uint32_t key = kb == 0 ? prev_x : (kb == 1 ? sl : sl + kTile);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
             const uint64_t a = smem_desc(sl + ks * 32, 16, 1024);
-            const uint64_t bd = smem_desc(keys[kb] + ks * 32, 16, 1024);
+            const uint64_t bd = smem_desc(key + ks * 32, 16, 1024);
             mma_ss(d + kb * 64, a, bd, idesc_s, ks > 0 ? 1u : 0u);
           }
         }
         mma_commit(&bar->s_full[b]);
         return true;
       };
-      if (have_cur) ok = issue_s(cur, 0);
+      if (have_cur) {
+        if (cur.first && cur.p > 0) cur_pre = pre_uses++ % kPre;
+        ok = issue_s(cur, 0, cur_pre);
+      }
       while (have_cur && ok) {
         const bool have_nxt = it.next(nxt);
-        if (have_nxt && !issue_s(nxt, n + 1)) break;
+        nxt_pre = -1;
+        if (have_nxt && nxt.first && nxt.p > 0) nxt_pre = pre_uses++ % kPre;
+        if (have_nxt && !issue_s(nxt, n + 1, nxt_pre)) break;
         // O = P V for job n
-        if (!mbar_wait(&bar->p_full, (uint32_t)n & 1u, abort, status)) break;
-        if (n >= 2 && !mbar_wait(&bar->o_free[n & 1], (uint32_t)(n / 2 - 1) & 1u, abort, status))
+        const int b = n & 1;
+        if (!mbar_wait(&bar->p_full[b], (uint32_t)(n / 2) & 1u, abort, status)) break;
+        if (n >= 2 && !mbar_wait(&bar->o_free[b], (uint32_t)(n / 2 - 1) & 1u, abort, status))
           break;
         tc_fence_after();
         const int s = n % kSlots;
         const uint32_t sl = slots_a + s * kSlotBytes;
         const bool has_prev = cur.p > 0, has_odd = 2 * cur.p + 1 < n_chunks;
-        const uint32_t prev_v = cur.first
-                                    ? pre_a + kTile
+        const uint32_t prev_v = cur_pre >= 0
+                                    ? pres_a + cur_pre * kPreBytes + kTile
                                     : slots_a + ((n + kSlots - 1) % kSlots) * kSlotBytes + 3 * kTile;
-        const uint32_t vals[3] = {prev_v, sl + 2 * kTile, sl + 3 * kTile};
-        const uint32_t d = tmem + 2 * kSCols + (uint32_t)(n & 1) * 64;
+        const uint32_t d = tmem + kOCol + (uint32_t)b * 64;
+        const uint32_t pa = tmem + (uint32_t)b * kSCols;
         bool acc = false;
+#pragma unroll
         for (int kb = 0; kb < 3; ++kb) {
           if ((kb == 0 && !has_prev) || (kb == 2 && !has_odd)) continue;
+          const uint32_t val = kb == 0 ? prev_v : (kb == 1 ? sl + 2 * kTile : sl + 3 * kTile);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t a = smem_desc(p_a + kb * (128 * 128) + ks * 32, 16, 1024);
-            const uint64_t bd = smem_desc(vals[kb] + ks * 2048, 8192, 1024);
-            mma_ss(d, a, bd, idesc_o, acc ? 1u : 0u);
+            const uint64_t bd = smem_desc(val + ks * 2048, 8192, 1024);
+            mma_ts(d, pa + kb * 32 + ks * 8, bd, idesc_o, acc ? 1u : 0u);
             acc = true;
           }
         }
-        mma_commit(&bar->p_free);                       // P consumed, O(n) ready
+        mma_commit(&bar->p_free[b]);                    // P(n) consumed, O(n) ready
         if (n >= 1) mma_commit(&bar->slot_free[(n - 1) % kSlots]);
-        if (cur.first && cur.p > 0) mma_commit(&bar->pre_free);
+        if (cur_pre >= 0) mma_commit(&bar->pre_free[cur_pre]);
         cur = nxt;
+        cur_pre = nxt_pre;
         have_cur = have_nxt;
         ++n;
       }
@@ -295,142 +362,138 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
       mbar_wait(&bar->mma_done, 0, (volatile int*)&dummy, status);
     }
   } else {
-    // ------------------------------------------------ softmax + epilogue
+    // ------------------------------------------------ softmax warpgroups
+    const int wg = (warp - 5) >> 2;             // 0: even jobs, 1: odd jobs
     const int q = warp & 3;                     // TMEM lane quarter (rows 32q..32q+31)
     const int row = q * 32 + lane;              // query row in the pair tile
     const bool odd_row = row >= 64;             // row belongs to chunk 2p+1
     const int kb0 = odd_row ? 1 : 0;            // first key block of this row
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t sbuf = tmem + lane_off + (uint32_t)wg * kSCols;
+    const uint32_t obuf = tmem + lane_off + kOCol + (uint32_t)wg * 64;
     JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
     Job j;
-    int n = 0;
-    // pending epilogue state of the previous job
+    int n = 0, pre_uses = 0;
     bool pend = false, pend_write = false;
     float pend_inv_l = 0.f, pend_lse = 0.f;
     int64_t pend_row = 0;
-    auto epilogue = [&](int nn) {
-      // O(nn) is complete (p_free phase nn observed by the caller)
+    int pend_n = 0;
+    auto epilogue = [&]() {
+      // O of this warpgroup's previous job is complete once its PV is done
+      if (!mbar_wait(&bar->p_free[wg], (uint32_t)(pend_n / 2) & 1u, abort, status)) return false;
       tc_fence_after();
-      const uint32_t taddr =
-          tmem + ((uint32_t)(q * 32) << 16) + 2 * kSCols + (uint32_t)(nn & 1) * 64;
-      uint32_t o0[32], o1[32];
-      tmem_ld32(taddr, o0);
-      tmem_ld32(taddr + 32, o1);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&bar->o_free[nn & 1]);
-      if (pend_write) {
-        uint4* dst = reinterpret_cast<uint4*>(opart + pend_row * 64);
+      uint4* dst = reinterpret_cast<uint4*>(opart + pend_row * 64);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint4 w;
-          __half2 h0 = __floats2half2_rn(__uint_as_float(o0[8 * c + 0]) * pend_inv_l,
-                                         __uint_as_float(o0[8 * c + 1]) * pend_inv_l);
-          __half2 h1 = __floats2half2_rn(__uint_as_float(o0[8 * c + 2]) * pend_inv_l,
-                                         __uint_as_float(o0[8 * c + 3]) * pend_inv_l);
-          __half2 h2 = __floats2half2_rn(__uint_as_float(o0[8 * c + 4]) * pend_inv_l,
-                                         __uint_as_float(o0[8 * c + 5]) * pend_inv_l);
-          __half2 h3 = __floats2half2_rn(__uint_as_float(o0[8 * c + 6]) * pend_inv_l,
-                                         __uint_as_float(o0[8 * c + 7]) * pend_inv_l);
-          w.x = *reinterpret_cast<uint32_t*>(&h0); w.y = *reinterpret_cast<uint32_t*>(&h1);
-          w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
-          dst[c] = w;
+      for (int h = 0; h < 2; ++h) {
+        uint32_t o[32];
+        tmem_ld32(obuf + 32 * h, o);
+        tmem_ld_wait();
+        if (h == 1) {
+          tc_fence_before();
+          mbar_arrive(&bar->o_free[wg]);
         }
+        if (pend_write) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint4 w;
-          __half2 h0 = __floats2half2_rn(__uint_as_float(o1[8 * c + 0]) * pend_inv_l,
-                                         __uint_as_float(o1[8 * c + 1]) * pend_inv_l);
-          __half2 h1 = __floats2half2_rn(__uint_as_float(o1[8 * c + 2]) * pend_inv_l,
-                                         __uint_as_float(o1[8 * c + 3]) * pend_inv_l);
-          __half2 h2 = __floats2half2_rn(__uint_as_float(o1[8 * c + 4]) * pend_inv_l,
-                                         __uint_as_float(o1[8 * c + 5]) * pend_inv_l);
-          __half2 h3 = __floats2half2_rn(__uint_as_float(o1[8 * c + 6]) * pend_inv_l,
-                                         __uint_as_float(o1[8 * c + 7]) * pend_inv_l);
-          w.x = *reinterpret_cast<uint32_t*>(&h0); w.y = *reinterpret_cast<uint32_t*>(&h1);
-          w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
-          dst[4 + c] = w;
+          for (int c = 0; c < 4; ++c)
+            dst[4 * h + c] = make_uint4(pack_f16x2(__uint_as_float(o[8 * c + 0]) * pend_inv_l,
+                                                   __uint_as_float(o[8 * c + 1]) * pend_inv_l),
+                                        pack_f16x2(__uint_as_float(o[8 * c + 2]) * pend_inv_l,
+                                                   __uint_as_float(o[8 * c + 3]) * pend_inv_l),
+                                        pack_f16x2(__uint_as_float(o[8 * c + 4]) * pend_inv_l,
+                                                   __uint_as_float(o[8 * c + 5]) * pend_inv_l),
+                                        pack_f16x2(__uint_as_float(o[8 * c + 6]) * pend_inv_l,
+                                                   __uint_as_float(o[8 * c + 7]) * pend_inv_l));
         }
-        lsepart[pend_row] = pend_lse;
       }
+      if (pend_write) lsepart[pend_row] = pend_lse;
+      return true;
     };
     bool ok = true;
     while (ok && it.next(j)) {
-      const int b = n & 1, s = n % kSlots;
-      if (!mbar_wait(&bar->s_full[b], (uint32_t)(n / 2) & 1u, abort, status)) break;
+      const bool use_pre = j.first && j.p > 0;
+      const int pb = use_pre ? pre_uses++ % kPre : -1;
+      if ((n & 1) != wg) { ++n; continue; }
+      if (pend && !epilogue()) break;
+      pend = false;
+      const int s = n % kSlots;
+      if (!mbar_wait(&bar->s_full[wg], (uint32_t)(n / 2) & 1u, abort, status)) break;
       tc_fence_after();
-      // S row: 128 columns starting at key block kb0
-      uint32_t sv[128];
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)b * kSCols + kb0 * 64;
-      tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-      tmem_ld32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&bar->s_free[b]);
       const bool has_prev = j.p > 0, has_odd = 2 * j.p + 1 < n_chunks;
       const bool row_live = !odd_row || has_odd;
       const int qpos = bar->kpos[s][row];
-      const int* kp_lo = (kb0 == 0) ? (j.first ? bar->kpos_pre
-                                               : bar->kpos[(n + kSlots - 1) % kSlots] + 64)
-                                    : bar->kpos[s];
-      const int* kp_hi = (kb0 == 0) ? bar->kpos[s] : bar->kpos[s] + 64;
-      const bool lo_ok = (kb0 == 0) ? has_prev : true;
+      const int* kp_lo = kb0 == 0 ? (pb >= 0 ? bar->kpos_pre[pb]
+                                             : bar->kpos[(n + kSlots - 1) % kSlots] + 64)
+                                  : bar->kpos[s];
+      const int* kp_hi = kb0 == 0 ? bar->kpos[s] : bar->kpos[s] + 64;
+      const bool lo_ok = kb0 == 0 ? has_prev : true;
+      // pass 1: mask and row max over this row's 128 keys; masked values
+      // (-inf) are written back so pass 2 needs no positions
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const int kp = (c < 64) ? kp_lo[c] : kp_hi[c - 64];
-        const bool blk_ok = (c < 64) ? lo_ok : true;
-        const bool valid = blk_ok && (causal ? (kp < qpos) : (kp != qpos));
-        const float x = valid ? __uint_as_float(sv[c]) * scale_log2 : -INFINITY;
-        sv[c] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
-      }
-      const float ms = (mx == -INFINITY) ? 0.f : mx;
-      // P buffer is free once PV(n-1) is done; that also completes O(n-1)
-      if (n >= 1 && !mbar_wait(&bar->p_free, (uint32_t)(n - 1) & 1u, abort, status)) break;
-      // P row: key blocks kb0 and kb0+1 hold exp2(s - max), the third block is 0
-      float l = 0.f;
-      uint8_t* prow = pbuf + row * 128;
-      const uint32_t sw = (uint32_t)(row & 7);
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const uint32_t col = (uint32_t)(kb0 * 64 + c4 * 32);
+        uint32_t sv[32];
+        tmem_ld32(sbuf + col, sv);
+        tmem_ld_wait();
+        const int* kp = (c4 < 2) ? kp_lo + c4 * 32 : kp_hi + (c4 - 2) * 32;
+        const bool blk_ok = (c4 < 2) ? lo_ok : true;
 #pragma unroll
-      for (int g = 0; g < 16; ++g) {             // 16 groups of 8 columns
-        uint32_t w[4];
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const int4 k4 = blk_ok ? *reinterpret_cast<const int4*>(kp + 4 * i4)
+                                 : make_int4(0, 0, 0, 0);
+          const int kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float e0 = ex2(__uint_as_float(sv[8 * g + 2 * e]) - ms);
-          const float e1 = ex2(__uint_as_float(sv[8 * g + 2 * e + 1]) - ms);
-          l += e0 + e1;
-          __half2 h = __floats2half2_rn(e0, e1);
-          w[e] = *reinterpret_cast<uint32_t*>(&h);
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * i4 + e;
+            const bool valid = blk_ok && (kCausal ? (kk[e] < qpos) : (kk[e] != qpos));
+            const float x = valid ? __uint_as_float(sv[i]) : -INFINITY;
+            sv[i] = __float_as_uint(x);
+            mx = fmaxf(mx, x);
+          }
         }
-        const int blk = kb0 + (g >> 3), ch = g & 7;
-        *reinterpret_cast<uint4*>(prow + blk * (128 * 128) + (((uint32_t)ch ^ sw) << 4)) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+        tmem_st32(sbuf + col, sv);
+      }
+      tmem_st_wait();
+      const bool has = mx != -INFINITY;
+      const float neg = has ? -mx * scale_log2 : 0.f;
+      // pass 2: P = exp2(scale * (s - max)) as fp16 pairs into TMEM over S;
+      // P column block kb lives at TMEM columns [32 kb, 32 kb + 32)
+      float l = 0.f;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t sv[32];
+        tmem_ld32(sbuf + (uint32_t)(kb0 * 64 + c4 * 32), sv);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float e0 = ex2(fmaf(__uint_as_float(sv[2 * e]), scale_log2, neg));
+          const float e1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), scale_log2, neg));
+          l += e0 + e1;
+          pk[e] = pack_f16x2(e0, e1);
+        }
+        tmem_st16(sbuf + (uint32_t)(kb0 * 32 + c4 * 16), pk);
       }
       {
-        const int zblk = odd_row ? 0 : 2;
+        uint32_t z[32];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          *reinterpret_cast<uint4*>(prow + zblk * (128 * 128) + (((uint32_t)ch ^ sw) << 4)) =
-              make_uint4(0u, 0u, 0u, 0u);
+        for (int e = 0; e < 32; ++e) z[e] = 0u;
+        tmem_st32(sbuf + (uint32_t)(odd_row ? 0 : 64), z);
       }
-      fence_proxy_async();
-      mbar_arrive(&bar->p_full);
-      if (pend) epilogue(n - 1);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bar->p_full[wg]);
       pend = true;
+      pend_n = n;
       pend_write = row_live;
       const int64_t bh = j.seg / n_rounds;
       const int r = (int)(j.seg % n_rounds);
       pend_row = (int64_t)r * N + bh * L + qpos;
-      const bool has = mx != -INFINITY;
       pend_inv_l = has ? 1.f / l : 0.f;
-      pend_lse = has ? (mx + log2f(l)) * kLn2 : -INFINITY;
+      pend_lse = has ? (mx * scale_log2 + log2f(l)) * kLn2 : -INFINITY;
       ++n;
     }
-    if (ok && pend && !*abort) {
-      if (mbar_wait(&bar->p_free, (uint32_t)(n - 1) & 1u, abort, status)) epilogue(n - 1);
-    }
+    if (pend && !*abort) epilogue();
   }
   tc_fence_before();
   __syncthreads();
@@ -442,14 +505,10 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
 
 }  // namespace
 
-size_t fwd_tc_partial_bytes(const lsh_problem& p) {
-  return (size_t)p.n_rounds * p.B * p.H * p.L * 64 * sizeof(__half);
-}
-
 cudaError_t launch_attn_fwd_tc(const lsh_problem& p, const void* qk, const void* v,
                                const int32_t* perm, void* opart_f16, float* lsepart, int* status,
                                cudaStream_t s) {
-  if (p.dtype != LSH_BF16 || p.chunk != kM) return cudaErrorNotSupported;
+  if (p.dtype != LSH_BF16 || p.chunk != kM || !(p.scale > 0.f)) return cudaErrorNotSupported;
   const int n_chunks = p.L / kM;
   const int n_pairs = (n_chunks + 1) / 2;
   const int units_per_seg = (n_pairs + kUnit - 1) / kUnit;
@@ -458,12 +517,13 @@ cudaError_t launch_attn_fwd_tc(const lsh_problem& p, const void* qk, const void*
   const int64_t N = (int64_t)p.B * p.H * p.L;
   int grid = sm_count();
   if ((int64_t)grid > n_units) grid = (int)n_units;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  auto kern = p.causal ? attn_fwd_tc_kernel<true> : attn_fwd_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  attn_fwd_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(
-      (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, perm, (__half*)opart_f16, lsepart, p.L,
-      p.n_rounds, N, p.causal, p.scale * kLog2e, n_units, units_per_seg, status);
+  kern<<<grid, kThreads, kSmemBytes, s>>>((const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, perm,
+                                          (__half*)opart_f16, lsepart, p.L, p.n_rounds, N,
+                                          p.scale * kLog2e, n_units, units_per_seg, status);
   note_launch();
   return cudaGetLastError();
 }

@@ -170,8 +170,14 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     int job = 0;
     bool ok = true;
     for (int t = ci; t < n_tiles && ok; t += ctas_per_round) {
-      float best_v = 0.f;
-      int best_c = 0;
+      // 32 independent running maxima, one per column position within a
+      // 32-column group (no serial dependency between columns); acc_g[i] is
+      // the group whose column i holds the best |s| so far (first on ties).
+      float acc[32];
+      int acc_g[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) { acc[i] = 0.f; acc_g[i] = 0; }
+      int g = 0;                              // global 32-column group index
       for (int j = 0; j < nsub; ++j, ++job) {
         const int buf = job & 1;
         if (!mbar_wait(&bar->acc_full[buf], (uint32_t)(job >> 1) & 1u, abort, status)) {
@@ -181,17 +187,25 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         tc_fence_after();
         const int ncols = min(kChunkN, nh - j * kChunkN);
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kChunkN);
-        for (int c0 = 0; c0 < ncols; c0 += 32) {
+        for (int c0 = 0; c0 < ncols; c0 += 32, ++g) {
           uint32_t v[32];
           tmem_ld32(taddr + c0, v);
           tmem_ld_wait();
-          const int cbase = j * kChunkN + c0;
+          if (c0 + 32 <= ncols) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float x = __uint_as_float(v[i]);
-            if (c0 + i < ncols && fabsf(x) > fabsf(best_v)) {
-              best_v = x;
-              best_c = cbase + i;
+            for (int i = 0; i < 32; ++i) {
+              const float x = __uint_as_float(v[i]);
+              const bool gt = fabsf(x) > fabsf(acc[i]);
+              acc[i] = gt ? x : acc[i];
+              acc_g[i] = gt ? g : acc_g[i];
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float x = __uint_as_float(v[i]);
+              const bool gt = (c0 + i < ncols) && fabsf(x) > fabsf(acc[i]);
+              acc[i] = gt ? x : acc[i];
+              acc_g[i] = gt ? g : acc_g[i];
             }
           }
         }
@@ -199,6 +213,15 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         mbar_arrive(&bar->acc_empty[buf]);
       }
       if (!ok) break;
+      // merge: largest |s|, smallest column on ties
+      float best_v = acc[0];
+      int best_c = acc_g[0] * 32;
+#pragma unroll
+      for (int i = 1; i < 32; ++i) {
+        const int c = acc_g[i] * 32 + i;
+        const float a = fabsf(acc[i]), b = fabsf(best_v);
+        if (a > b || (a == b && c < best_c)) { best_v = acc[i]; best_c = c; }
+      }
       const int64_t row = (int64_t)t * kTileM + row_in_tile;
       if (row < n_rows) {
         const int64_t bh = row / L, pos = row - bh * L;
