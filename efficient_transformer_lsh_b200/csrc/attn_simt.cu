@@ -411,10 +411,13 @@ cudaError_t bwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* 
   if (e != cudaSuccess) return e;
   bwd_prep_kernel<T><<<(unsigned)((N * 16 + 255) / 256), 256, 0, s>>>(out, out_lo, dout, lse, D, dqk, dv,
                                                                         N);
+  note_launch();
+  e = launch_attn_bwd_tc(p, qk, v, dout, perm, lse, D, dqk, dv, status, s);
+  if (e != cudaErrorNotSupported) return e == cudaSuccess ? cudaGetLastError() : e;
   bwd_round_kernel<T><<<(unsigned)blocks, 256, kBwdSmem, s>>>(
       qk, v, dout, perm, lse, D, dqk, dv, p.L, p.chunk, p.n_rounds, p.causal, p.scale,
       p.scale * kLog2e, status);
-  note_launch(2);
+  note_launch();
   return cudaGetLastError();
 }
 
