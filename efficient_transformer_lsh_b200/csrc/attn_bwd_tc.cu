@@ -30,8 +30,12 @@
 //              chunks) into a 2-slot ring, in-place bf16 -> fp16 conversion,
 //              per-query position, log2-scaled LSE and D;
 //   warp 4   : TMEM allocation and the MMA-issuing thread;
-//   warps 5-8: one thread per key row: masks, P, dS (fp16), then the
-//              gradient epilogue with atomics.
+//   warps 5-8 and 9-12: two warpgroups, one thread per key row in each; the
+//              first takes the row's first query block, the second its second
+//              (P and dS are elementwise once LSE and D are known, so the two
+//              halves need no exchange); then the gradient epilogue with
+//              atomics, dV and R1 from the first warpgroup, dK + R0 from the
+//              second.
 #include <cuda_fp16.h>
 #include <stddef.h>
 
@@ -54,11 +58,17 @@ constexpr int kX = 0, kV = 3 * kTile, kDo = 5 * kTile;
 constexpr int kSlotBytes = 8 * kTile;  // 64 KB
 constexpr int kDsBlock = 128 * 128;    // 128 key rows x 64 query columns
 constexpr int kDsBytes = 4 * kDsBlock; // dS^T blocks 0,1,2 + a zero block
-constexpr int kThreads = 288;
+constexpr int kThreads = 416;
 // TMEM columns
-constexpr uint32_t kColS = 0, kColDp = 192;      // S^T, dP^T (P^T packed over S^T)
-constexpr uint32_t kColDv = 96, kColDk = 288;    // free halves after packing
+constexpr uint32_t kColS = 0, kColDp = 192;      // S^T, dP^T
+constexpr uint32_t kColDv = 96, kColDk = 288;    // accumulators in their upper halves
 constexpr uint32_t kColR0 = 384, kColR1 = 448;
+// P^T (fp16 pairs, 3 x 32 columns) lives in the R0/R1 columns while they are
+// idle: written after the previous item's flush, read by the dV MMAs, which
+// run before the R0/R1 MMAs that overwrite it (MMAs complete in issue order).
+// The S^T/dP^T columns are read by both key-row warpgroups, so nothing is
+// written there before both have read them.
+constexpr uint32_t kColP = 384;
 
 struct __align__(16) BwdBar {
   uint64_t slot_full[kSlots];
@@ -87,14 +97,14 @@ struct Job {
 };
 
 struct JobIter {
-  int64_t unit, n_units, stride;
+  int unit, n_units, stride;
   int units_per_seg, n_pairs, k;
-  __device__ JobIter(int64_t u0, int64_t nu, int64_t st, int ups, int np)
+  __device__ JobIter(int u0, int nu, int st, int ups, int np)
       : unit(u0), n_units(nu), stride(st), units_per_seg(ups), n_pairs(np), k(0) {}
   __device__ bool next(Job& j) {
     while (unit < n_units) {
-      const int64_t seg = unit / units_per_seg;
-      const int p0 = (int)(unit % units_per_seg) * kUnit;
+      const int seg = unit / units_per_seg;
+      const int p0 = (unit - seg * units_per_seg) * kUnit;
       const int p = p0 + k;
       if (k < kUnit && p < n_pairs) {
         j.seg = seg;
@@ -144,29 +154,42 @@ __device__ __forceinline__ void convert_row(uint8_t* tile, int row, int half) {
   }
 }
 
-// Adds scale * (64 consecutive TMEM columns of this lane [+ another 64]) to a
-// 64-float row of global memory with 16 vector atomics.
-__device__ __forceinline__ void flush_row(float* dst, uint32_t ta, uint32_t tb, bool two,
-                                          float scale, bool live) {
+// Adds scale * (64 consecutive TMEM columns of each lane [+ another 64]) to
+// the 64-float global row `row_of_lane` of that lane (token `tok`, or none
+// when tok < 0). The warp stages its 32 half-rows in shared memory and
+// re-reads them so that each vector atomic instruction covers four whole
+// 128-byte lines (8 lanes per row) instead of 32 scattered 16-byte pieces.
+constexpr int kStageStride = 144;   // bytes per staged half-row (128 + 16 pad)
+__device__ __forceinline__ void flush_rows(float* base, int tok, uint32_t ta, uint32_t tb,
+                                           bool two, float scale, uint8_t* stage, int lane) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     uint32_t a[32], b[32];
     tmem_ld32(ta + 32 * h, a);
     if (two) tmem_ld32(tb + 32 * h, b);
     tmem_ld_wait();
-    if (live) {
+    uint8_t* mine = stage + lane * kStageStride;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float x[4];
+    for (int c = 0; c < 8; ++c) {
+      float x[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float val = __uint_as_float(a[4 * c + e]);
-          if (two) val += __uint_as_float(b[4 * c + e]);
-          x[e] = val * scale;
-        }
-        red_add_v4(dst + 32 * h + 4 * c, x[0], x[1], x[2], x[3]);
+      for (int e = 0; e < 4; ++e) {
+        float val = __uint_as_float(a[4 * c + e]);
+        if (two) val += __uint_as_float(b[4 * c + e]);
+        x[e] = val * scale;
       }
+      *reinterpret_cast<float4*>(mine + 16 * c) = make_float4(x[0], x[1], x[2], x[3]);
     }
+    __syncwarp();
+    const int piece = lane & 7;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int r = 4 * k + (lane >> 3);
+      const int rt = __shfl_sync(0xffffffffu, tok, r);
+      const float4 val = *reinterpret_cast<const float4*>(stage + r * kStageStride + 16 * piece);
+      if (rt >= 0) red_add_v4(base + (int64_t)rt * 64 + 32 * h + 4 * piece, val.x, val.y, val.z, val.w);
+    }
+    __syncwarp();
   }
 }
 
@@ -176,12 +199,13 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
                    const __nv_bfloat16* __restrict__ dout, const int32_t* __restrict__ perm,
                    const float* __restrict__ lse, const float* __restrict__ Dg,
                    float* __restrict__ dqk, float* __restrict__ dv, int L, int n_rounds,
-                   float scale, float scale_log2, int64_t n_units, int units_per_seg,
+                   float scale, float scale_log2, int n_units, int units_per_seg,
                    int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* slots = smem;
   uint8_t* dsb = slots + kSlots * kSlotBytes;
+  static_assert(8 * 32 * kStageStride <= 3 * kDsBlock, "flush staging fits in the dS^T blocks");
   BwdBar* bar = (BwdBar*)(dsb + kDsBytes);
   volatile int* abort = &bar->abort;
 
@@ -195,9 +219,9 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
       mbar_init(&bar->slot_free[s], 1);
     }
     mbar_init(&bar->s_full, 1);
-    mbar_init(&bar->p_full, 128);
+    mbar_init(&bar->p_full, 256);
     mbar_init(&bar->g_full, 1);
-    mbar_init(&bar->g_free, 128);
+    mbar_init(&bar->g_free, 256);
     mbar_init(&bar->mma_done, 1);
     bar->abort = 0;
     fence_mbar_init();
@@ -322,7 +346,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
             // dV += P^T (TMEM) . dO_Q ; dK += dS^T (smem, K-major) . X_Q
-            mma_ts(tmem + kColDv, tmem + kColS + qb * 32 + ks * 8,
+            mma_ts(tmem + kColDv, tmem + kColP + qb * 32 + ks * 8,
                    smem_desc(sl + kDo + qb * kTile + ks * 2048, 8192, 1024), idesc_kn, acc_v);
             acc_v = true;
             mma_ss(tmem + kColDk, smem_desc(ds_a + qb * kDsBlock + ks * 32, 16, 1024),
@@ -349,6 +373,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
     }
   } else {
     // ------------------------------------------------ key rows: P, dS, gradients
+    const int kwg = (warp - 5) >> 2;           // 0: first query block, 1: second
     const int q = warp & 3;
     const int row = q * 32 + lane;             // key row = TMEM lane
     const bool odd_row = row >= 64;
@@ -371,9 +396,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
       const int* qp_all = bar->qpos[s];
       const float* l2_all = bar->lse2[s];
       const float* d_all = bar->dval[s];
-#pragma unroll
-      for (int bi = 0; bi < 2; ++bi) {
-        const int qb = qb0 + bi;
+      {
+        const int qb = qb0 + kwg;
         const bool blk_ok = qb < nc && row_live;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -409,8 +433,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
             dk[2 * i4] = pack_f16x2(de[0], de[1]);
             dk[2 * i4 + 1] = pack_f16x2(de[2], de[3]);
           }
-          // P^T into TMEM over S^T (block qb at columns 32 qb), dS^T into smem
-          tmem_st16(tl + kColS + (uint32_t)(qb * 32 + h * 16), pk);
+          // P^T into TMEM (block qb at columns kColP + 32 qb), dS^T into smem
+          tmem_st16(tl + kColP + (uint32_t)(qb * 32 + h * 16), pk);
           uint8_t* drow = dsb + qb * kDsBlock + row * 128;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -420,13 +444,13 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
           }
         }
       }
-      {
+      if (kwg == 1) {
         // the query block this key row does not see: P = 0 and dS = 0
         const int zb = odd_row ? 0 : 2;
         uint32_t z[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) z[e] = 0u;
-        tmem_st32(tl + kColS + (uint32_t)(zb * 32), z);
+        tmem_st32(tl + kColP + (uint32_t)(zb * 32), z);
         uint8_t* drow = dsb + zb * kDsBlock + row * 128;
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch)
@@ -440,13 +464,16 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
       if (!mbar_wait(&bar->g_full, (uint32_t)n & 1u, abort, status)) break;
       tc_fence_after();
       const int64_t bh = j.seg / n_rounds;
-      float* dv_row = dv + (bh * L + kpos) * 64;
-      float* dx_row = dqk + (bh * L + kpos) * 64;
-      flush_row(dv_row, tl + kColDv, 0, false, 1.f, row_live);
-      flush_row(dx_row, tl + kColDk, tl + kColR0, true, scale, row_live);
-      if (nc == 3 && !odd_row) {
+      // staging: the dS^T blocks are idle until the next item's softmax,
+      // which starts only after every row here has been flushed
+      uint8_t* stage = dsb + (warp - 5) * (32 * kStageStride);
+      const int tok = row_live ? kpos : -1;
+      if (kwg == 0) flush_rows(dv + bh * L * 64, tok, tl + kColDv, 0, false, 1.f, stage, lane);
+      if (kwg == 1)
+        flush_rows(dqk + bh * L * 64, tok, tl + kColDk, tl + kColR0, true, scale, stage, lane);
+      if (kwg == 0 && nc == 3 && !odd_row) {
         // query-side term of chunk 2p+2 (lanes 0..63 of R1)
-        flush_row(dqk + (bh * L + qpos2) * 64, tl + kColR1, 0, false, scale, true);
+        flush_rows(dqk + bh * L * 64, qpos2, tl + kColR1, 0, false, scale, stage, lane);
       }
       tc_fence_before();
       mbar_arrive(&bar->g_free);
@@ -471,6 +498,7 @@ cudaError_t launch_attn_bwd_tc(const lsh_problem& p, const void* qk, const void*
   const int n_pairs = (n_chunks + 1) / 2;
   const int units_per_seg = (n_pairs + kUnit - 1) / kUnit;
   const int64_t n_units = (int64_t)p.B * p.H * p.n_rounds * units_per_seg;
+  if (n_units > INT32_MAX) return cudaErrorNotSupported;
   int grid = sm_count();
   if ((int64_t)grid > n_units) grid = (int)n_units;
   auto kern = p.causal ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
@@ -479,7 +507,7 @@ cudaError_t launch_attn_bwd_tc(const lsh_problem& p, const void* qk, const void*
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemBytes, s>>>(
       (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, (const __nv_bfloat16*)dout, perm, lse, D,
-      dqk, dv, p.L, p.n_rounds, p.scale, p.scale * kLog2e, n_units, units_per_seg, status);
+      dqk, dv, p.L, p.n_rounds, p.scale, p.scale * kLog2e, (int)n_units, units_per_seg, status);
   note_launch();
   return cudaGetLastError();
 }

@@ -16,10 +16,12 @@
 // (batch, head, round) segment):
 //   warps 0-3  : producers — cp.async gathers of x and v rows through perm
 //                straight into the 128-byte-swizzled K-major layout of a
-//                4-slot ring (a unit's first pair also needs chunk 2p0-1,
+//                5-slot ring (a unit's first pair also needs chunk 2p0-1,
 //                which goes to one of 3 rotating side buffers); each thread
-//                then converts its own pieces bf16 -> fp16 in place (exact
-//                for |values| < 65504). Software-pipelined one job deep;
+//                then converts its own pieces of v bf16 -> fp16 in place
+//                (exact for |values| < 65504); x stays bf16, whose products
+//                are exact in the Q K^T MMA too. Software-pipelined one job
+//                deep, with the next job's perm entries loaded a job ahead;
 //   warp 4     : TMEM allocation; one thread issues S = Q K^T (three
 //                128x64x64 MMAs per pair into a double-buffered TMEM S) and
 //                O = P V with P read from TMEM (A operand) and V from shared
@@ -47,7 +49,7 @@ using namespace tc;
 
 constexpr int kM = 64;            // chunk
 constexpr int kUnit = 8;          // pairs per work unit
-constexpr int kSlots = 4;         // pair slots in the ring
+constexpr int kSlots = 5;         // pair slots in the ring
 constexpr int kPre = 3;           // side buffers for a unit's previous chunk
 constexpr int kTile = 64 * 128;   // one chunk of 64 rows x 64 16-bit values = 8 KB
 constexpr int kSlotBytes = 4 * kTile;   // x_even | x_odd | v_even | v_odd
@@ -85,14 +87,14 @@ struct Job {
 
 // Walks the CTA's units in order; every role iterates the same sequence.
 struct JobIter {
-  int64_t unit, n_units, stride;
+  int unit, n_units, stride;
   int units_per_seg, n_pairs, k;
-  __device__ JobIter(int64_t u0, int64_t nu, int64_t st, int ups, int np)
+  __device__ JobIter(int u0, int nu, int st, int ups, int np)
       : unit(u0), n_units(nu), stride(st), units_per_seg(ups), n_pairs(np), k(0) {}
   __device__ bool next(Job& j) {
     while (unit < n_units) {
-      const int64_t seg = unit / units_per_seg;
-      const int p = (int)(unit % units_per_seg) * kUnit + k;
+      const int seg = unit / units_per_seg;
+      const int p = (unit - seg * units_per_seg) * kUnit + k;
       if (k < kUnit && p < n_pairs) {
         j.seg = seg;
         j.p = p;
@@ -119,18 +121,6 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return r;
 }
 
-// Position of row `row` of chunk c, checked against L (a bad id is recorded
-// in the status word and replaced by 0 so no copy leaves the tensor).
-__device__ __forceinline__ int chunk_pos(const int32_t* __restrict__ perm, int64_t seg, int L, int c,
-                                         int row, int* status) {
-  int pos = perm[seg * L + (int64_t)c * kM + row];
-  if ((unsigned)pos >= (unsigned)L) {
-    if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
-    pos = 0;
-  }
-  return pos;
-}
-
 // Thread t copies 16-byte pieces 4*(t&1)..+3 of row t>>1 of a chunk tile into
 // their 128-byte-swizzled places (bf16; converted later in place).
 __device__ __forceinline__ void issue_row(const __nv_bfloat16* __restrict__ src_row, uint8_t* tile,
@@ -155,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __restrict__ v,
                    const int32_t* __restrict__ perm, __half* __restrict__ opart,
                    float* __restrict__ lsepart, int L, int n_rounds, int64_t N, float scale_log2,
-                   int64_t n_units, int units_per_seg, int* status) {
+                   int n_units, int units_per_seg, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* slots = smem;
@@ -198,11 +188,21 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
     JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
     Job cur, nxt;
     bool have_cur = it.next(cur);
+    // perm entries of the next job are loaded one iteration ahead and only
+    // checked when used, so the loads overlap the rest of the iteration
     int pos_p = 0, pos_e = 0, pos_o = 0;
     auto fetch_pos = [&](const Job& jb) {
-      pos_e = chunk_pos(perm, jb.seg, L, 2 * jb.p, row, status);
-      pos_o = (2 * jb.p + 1 < n_chunks) ? chunk_pos(perm, jb.seg, L, 2 * jb.p + 1, row, status) : 0;
-      pos_p = (jb.first && jb.p > 0) ? chunk_pos(perm, jb.seg, L, 2 * jb.p - 1, row, status) : 0;
+      const int32_t* pr = perm + jb.seg * L + row;
+      pos_e = __ldg(pr + (int64_t)(2 * jb.p) * kM);
+      pos_o = (2 * jb.p + 1 < n_chunks) ? __ldg(pr + (int64_t)(2 * jb.p + 1) * kM) : 0;
+      pos_p = (jb.first && jb.p > 0) ? __ldg(pr + (int64_t)(2 * jb.p - 1) * kM) : 0;
+    };
+    auto checked = [&](int ps) {
+      if ((unsigned)ps >= (unsigned)L) {
+        if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
+        ps = 0;
+      }
+      return ps;
     };
     if (have_cur) fetch_pos(cur);
     int n = 0, pre_uses = 0;
@@ -211,17 +211,9 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
     bool ok = true;
     auto publish = [&]() {
       uint8_t* ps = slots + pend_slot * kSlotBytes;
-      if (pend_pre >= 0) {
-        uint8_t* pb = pres + pend_pre * kPreBytes;
-        convert_row(pb, row, half);
-        convert_row(pb + kTile, row, half);
-      }
-      convert_row(ps, row, half);
+      if (pend_pre >= 0) convert_row(pres + pend_pre * kPreBytes + kTile, row, half);
       convert_row(ps + 2 * kTile, row, half);
-      if (pend_odd) {
-        convert_row(ps + kTile, row, half);
-        convert_row(ps + 3 * kTile, row, half);
-      }
+      if (pend_odd) convert_row(ps + 3 * kTile, row, half);
       fence_proxy_async();
       mbar_arrive(&bar->slot_full[pend_slot]);
     };
@@ -245,6 +237,9 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
         ++pre_uses;
       }
       const int64_t bh = cur.seg / n_rounds;
+      pos_e = checked(pos_e);
+      pos_o = checked(pos_o);
+      pos_p = checked(pos_p);
       uint8_t* sl = slots + s * kSlotBytes;
       const __nv_bfloat16* xb = qk + bh * L * 64;
       const __nv_bfloat16* vb = v + bh * L * 64;
@@ -281,7 +276,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
   } else if (warp == 4) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_f16(128, 64, 0, false, false);   // Q K^T, both K-major
+      const uint32_t idesc_s = idesc_f16(128, 64, 1, false, false);   // Q K^T: bf16, K-major
       const uint32_t idesc_o = idesc_f16(128, 64, 0, false, true);    // P V, V MN-major
       const uint32_t slots_a = smem_u32(slots), pres_a = smem_u32(pres);
       JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
@@ -515,6 +510,7 @@ cudaError_t launch_attn_fwd_tc(const lsh_problem& p, const void* qk, const void*
   const int64_t n_segs = (int64_t)p.B * p.H * p.n_rounds;
   const int64_t n_units = n_segs * units_per_seg;
   const int64_t N = (int64_t)p.B * p.H * p.L;
+  if (n_units > INT32_MAX) return cudaErrorNotSupported;
   int grid = sm_count();
   if ((int64_t)grid > n_units) grid = (int)n_units;
   auto kern = p.causal ? attn_fwd_tc_kernel<true> : attn_fwd_tc_kernel<false>;
@@ -523,7 +519,7 @@ cudaError_t launch_attn_fwd_tc(const lsh_problem& p, const void* qk, const void*
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemBytes, s>>>((const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, perm,
                                           (__half*)opart_f16, lsepart, p.L, p.n_rounds, N,
-                                          p.scale * kLog2e, n_units, units_per_seg, status);
+                                          p.scale * kLog2e, (int)n_units, units_per_seg, status);
   note_launch();
   return cudaGetLastError();
 }

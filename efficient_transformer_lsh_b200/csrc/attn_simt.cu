@@ -201,6 +201,93 @@ combine_kernel(const PT* __restrict__ opart, const float* __restrict__ lsepart,
   if (c4 == 0) lse[tok] = LSE;
 }
 
+// Round combine for fp16 per-round outputs (tensor-core forward): 8 threads
+// per token, 8 columns each (16-byte loads and stores); round loads are
+// unrolled so several are in flight.
+__device__ __forceinline__ void unpack8(uint4 u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+__device__ __forceinline__ uint4 pack8_bf16(const float* f) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__global__ void __launch_bounds__(256)
+combine_f16_kernel(const __half* __restrict__ opart, const float* __restrict__ lsepart,
+                   const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ out,
+                   __nv_bfloat16* __restrict__ out_lo, float* __restrict__ lse, int64_t N,
+                   int n_rounds) {
+  const int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
+  const int c8 = (threadIdx.x & 7) * 8;
+  if (tok >= N) return;
+  float mx = -INFINITY;
+  for (int r = 0; r < n_rounds; ++r) mx = fmaxf(mx, __ldg(lsepart + (int64_t)r * N + tok));
+  uint4* o16 = reinterpret_cast<uint4*>(out + tok * kD + c8);
+  if (mx == -INFINITY) {
+    *o16 = *reinterpret_cast<const uint4*>(v + tok * kD + c8);
+    if (out_lo) *reinterpret_cast<uint4*>(out_lo + tok * kD + c8) = make_uint4(0u, 0u, 0u, 0u);
+    if (c8 == 0) lse[tok] = -INFINITY;
+    return;
+  }
+  float tot = 0.f;
+  for (int r = 0; r < n_rounds; ++r) tot += __expf(__ldg(lsepart + (int64_t)r * N + tok) - mx);
+  const float LSE = mx + __logf(tot);
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  int r = 0;
+  for (; r + 4 <= n_rounds; r += 4) {
+    uint4 u[4];
+    float wgt[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      u[k] = __ldg(reinterpret_cast<const uint4*>(opart + ((int64_t)(r + k) * N + tok) * kD + c8));
+      const float l = __ldg(lsepart + (int64_t)(r + k) * N + tok);
+      wgt[k] = (l == -INFINITY) ? 0.f : __expf(l - LSE);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float f[8];
+      unpack8(u[k], f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(wgt[k], f[i], acc[i]);
+    }
+  }
+  for (; r < n_rounds; ++r) {
+    const float l = __ldg(lsepart + (int64_t)r * N + tok);
+    if (l == -INFINITY) continue;
+    float f[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(opart + ((int64_t)r * N + tok) * kD + c8)), f);
+    const float wgt = __expf(l - LSE);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = fmaf(wgt, f[i], acc[i]);
+  }
+  const uint4 hi = pack8_bf16(acc);
+  *o16 = hi;
+  if (out_lo) {
+    float lo[8];
+    const uint32_t w[4] = {hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      lo[2 * i] = acc[2 * i] - __uint_as_float(w[i] << 16);
+      lo[2 * i + 1] = acc[2 * i + 1] - __uint_as_float(w[i] & 0xffff0000u);
+    }
+    *reinterpret_cast<uint4*>(out_lo + tok * kD + c8) = pack8_bf16(lo);
+  }
+  if (c8 == 0) lse[tok] = LSE;
+}
+
 // D_i = dout_i . out_i; zero dqk; dv = dout for self-attending rows, else 0.
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -382,8 +469,10 @@ cudaError_t fwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* 
   const unsigned cblocks = (unsigned)((N * 16 + 255) / 256);
   cudaError_t e = launch_attn_fwd_tc(p, qk, v, perm, ws.opart, ws.lsepart, status, s);
   if (e == cudaSuccess) {
-    combine_kernel<T, __half><<<cblocks, 256, 0, s>>>((const __half*)ws.opart, ws.lsepart, v, out,
-                                                      out_lo, lse, N, p.n_rounds);
+    // the tensor-core forward handles bf16 problems only
+    combine_f16_kernel<<<(unsigned)((N * 8 + 255) / 256), 256, 0, s>>>(
+        (const __half*)ws.opart, ws.lsepart, (const __nv_bfloat16*)v, (__nv_bfloat16*)out,
+        (__nv_bfloat16*)out_lo, lse, N, p.n_rounds);
     note_launch();
     return cudaGetLastError();
   }

@@ -18,8 +18,13 @@
 //             accumulators (so the epilogue of one chunk overlaps the MMA of
 //             the next);
 //   warps 2-5: epilogue — tcgen05.ld of the accumulator rows (one token per
-//             thread), running max |s| with its column, bucket id written
-//             once per token.
+//             thread). Each |s| becomes a float key whose 4 low mantissa bits
+//             hold (15 - its 32-column group), so one 3-input max folds two
+//             columns into each of 32 per-position running maxima with the
+//             lowest column winning ties; values closer than 2^-19 relative
+//             count as ties (a near-tie by the 1e-5 bound the results are
+//             checked against). The winner's sign is recomputed from the X and
+//             R tiles in shared memory, then the bucket id is written.
 // Handles n_b/2 <= 512 with n_b/2 a multiple of 8; other shapes use the
 // CUDA-core kernel.
 #include "common.cuh"
@@ -75,7 +80,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     mbar_init(&bar->r_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar->x_full[s], 1);
-      mbar_init(&bar->x_empty[s], 1);
+      mbar_init(&bar->x_empty[s], 128);   // released by the epilogue (sign recompute)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar->acc_full[b], 1);
@@ -155,7 +160,6 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
             }
             mma_commit(&bar->acc_full[buf]);
           }
-          mma_commit(&bar->x_empty[s]);
         }
       }
       // all issued MMAs have finished before TMEM is released (bounded)
@@ -167,16 +171,12 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     // ---------------- epilogue: warps 2..5 ----------------
     const int q = warp & 3;                 // TMEM lane quarter this warp may read
     const int row_in_tile = q * 32 + lane;
-    int job = 0;
+    int job = 0, it = 0;
     bool ok = true;
-    for (int t = ci; t < n_tiles && ok; t += ctas_per_round) {
-      // 32 independent running maxima, one per column position within a
-      // 32-column group (no serial dependency between columns); acc_g[i] is
-      // the group whose column i holds the best |s| so far (first on ties).
+    for (int t = ci; t < n_tiles && ok; t += ctas_per_round, ++it) {
       float acc[32];
-      int acc_g[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) { acc[i] = 0.f; acc_g[i] = 0; }
+      for (int i = 0; i < 32; ++i) acc[i] = 0.f;
       int g = 0;                              // global 32-column group index
       for (int j = 0; j < nsub; ++j, ++job) {
         const int buf = job & 1;
@@ -187,45 +187,61 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         tc_fence_after();
         const int ncols = min(kChunkN, nh - j * kChunkN);
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kChunkN);
-        for (int c0 = 0; c0 < ncols; c0 += 32, ++g) {
-          uint32_t v[32];
-          tmem_ld32(taddr + c0, v);
+        for (int c0 = 0; c0 < ncols; c0 += 64, g += 2) {
+          uint32_t va[32], vb[32];
+          tmem_ld32(taddr + c0, va);
+          tmem_ld32(taddr + c0 + 32, vb);     // within the 512 allocated columns
           tmem_ld_wait();
-          if (c0 + 32 <= ncols) {
+          const uint32_t ma = (uint32_t)(15 - g), mb = (uint32_t)(14 - g);
+          const int na = min(32, ncols - c0), nb = min(32, ncols - c0 - 32);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float x = __uint_as_float(v[i]);
-              const bool gt = fabsf(x) > fabsf(acc[i]);
-              acc[i] = gt ? x : acc[i];
-              acc_g[i] = gt ? g : acc_g[i];
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float x = __uint_as_float(v[i]);
-              const bool gt = (c0 + i < ncols) && fabsf(x) > fabsf(acc[i]);
-              acc[i] = gt ? x : acc[i];
-              acc_g[i] = gt ? g : acc_g[i];
-            }
+          for (int i = 0; i < 32; ++i) {
+            const uint32_t ka = (i < na) ? ((va[i] & 0x7FFFFFF0u) | ma) : 0u;
+            const uint32_t kb = (i < nb) ? ((vb[i] & 0x7FFFFFF0u) | mb) : 0u;
+            float r;
+            asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(acc[i]), "f"(__uint_as_float(ka)),
+                "f"(__uint_as_float(kb)));
+            acc[i] = r;
           }
         }
         tc_fence_before();
         mbar_arrive(&bar->acc_empty[buf]);
       }
       if (!ok) break;
-      // merge: largest |s|, smallest column on ties
-      float best_v = acc[0];
-      int best_c = acc_g[0] * 32;
+      // merge: largest key magnitude, smallest column on ties
+      uint32_t best_m = 0;
+      int best_c = 0x7fffffff;
 #pragma unroll
-      for (int i = 1; i < 32; ++i) {
-        const int c = acc_g[i] * 32 + i;
-        const float a = fabsf(acc[i]), b = fabsf(best_v);
-        if (a > b || (a == b && c < best_c)) { best_v = acc[i]; best_c = c; }
+      for (int i = 0; i < 32; ++i) {
+        const uint32_t k = __float_as_uint(acc[i]);
+        const uint32_t m = k & 0x7FFFFFF0u;
+        const int c = (15 - (int)(k & 15u)) * 32 + i;
+        if (m > best_m || (m == best_m && c < best_c)) { best_m = m; best_c = c; }
       }
+      // sign of s at the winning column: x . R[:, col] from shared memory
+      const int s_idx = it % kStages;
+      const uint8_t* xrow = x_smem + s_idx * kXBytes + row_in_tile * 128;
+      const uint8_t* rblk = r_smem + (best_c >> 6) * kRBlockBytes;
+      const int nn = best_c & 63;
+      float dot = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 w = *reinterpret_cast<const uint4*>(xrow + (((uint32_t)c ^ (uint32_t)(row_in_tile & 7)) << 4));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int k = c * 8 + e;
+          const float xv = __uint_as_float((e & 1) ? (ws[e >> 1] & 0xffff0000u) : (ws[e >> 1] << 16));
+          const uint16_t rb = *reinterpret_cast<const uint16_t*>(
+              rblk + k * 128 + ((((uint32_t)nn >> 3) ^ (uint32_t)(k & 7)) << 4) + (nn & 7) * 2);
+          dot = fmaf(xv, __uint_as_float((uint32_t)rb << 16), dot);
+        }
+      }
+      mbar_arrive(&bar->x_empty[s_idx]);
       const int64_t row = (int64_t)t * kTileM + row_in_tile;
       if (row < n_rows) {
         const int64_t bh = row / L, pos = row - bh * L;
-        bucket[(bh * n_rounds + r) * L + pos] = best_v >= 0.f ? best_c : nh + best_c;
+        bucket[(bh * n_rounds + r) * L + pos] = dot >= 0.f ? best_c : nh + best_c;
       }
     }
   }

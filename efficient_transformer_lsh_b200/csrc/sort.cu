@@ -5,17 +5,24 @@
 // before chunking. Sorting stably by bucket is sorting by the packed key
 // (round, bucket, position), because positions arrive in increasing order.
 //
-// Counting sort in four passes over tiles of kTile positions:
-//   1. tile_sort: each tile sorts packed keys (bucket << 12 | local index) in
-//      shared memory (bitonic network), stores them, and records how many
-//      positions of each bucket it holds: counts[seg][bucket][tile];
+// Counting sort in four passes over tiles of positions:
+//   1. per tile, how many positions of each bucket it holds:
+//      counts[seg][bucket][tile]. For n_buckets <= 4096 (tiles of 2048) a
+//      warp walks 256 consecutive positions 32 at a time and counts with
+//      __match_any_sync into per-warp 16-bit counters; for larger bucket
+//      counts (tiles of 4096) the tile's packed keys (bucket << 12 | local
+//      index) are sorted in shared memory by a bitonic network and stored;
 //   2. row_scan: for every (seg, bucket), exclusive scan over tiles, plus the
 //      bucket total;
 //   3. bucket_scan: for every seg, exclusive scan of bucket totals;
-//   4. scatter: slot = base[seg][b] + counts[seg][b][tile] + rank within the
-//      tile's run of bucket b; perm[seg][slot] = position.
-// The packed local index makes every tile's order stable, and tiles are
-// placed in position order, so the whole sort is stable.
+//   4. scatter: slot = base[seg][b] + counts[seg][b][tile] + rank of the
+//      position among the tile's positions of bucket b; perm[seg][slot] =
+//      position. The warp path recomputes the ranks in position order (step
+//      by step, lanes in order, warps in order through an exclusive prefix
+//      of the per-warp counts); the bitonic path takes them from the sorted
+//      packed keys, whose local index breaks ties.
+// Ranks follow position order inside a tile and tiles are placed in position
+// order, so the whole sort is stable.
 #include "common.cuh"
 #include "internal.h"
 
@@ -174,12 +181,115 @@ scatter_kernel(const uint32_t* __restrict__ sorted, const int32_t* __restrict__ 
   }
 }
 
+// ---- warp-counting path (n_buckets <= kWarpMaxBuckets) --------------------
+constexpr int kWarpMaxBuckets = 4096;
+constexpr int kWarpsPerTile = 8;
+constexpr int kWarpKeys = 256;                        // positions per warp
+constexpr int kWTile = kWarpsPerTile * kWarpKeys;     // 2048 positions per tile
+constexpr size_t kWarpSmem = (size_t)kWarpsPerTile * kWarpMaxBuckets * 2 + kWarpMaxBuckets * 4;
+
+// Counts of each bucket among this warp's 256 positions into cnt[b] (16-bit).
+__device__ __forceinline__ void warp_count(const int32_t* __restrict__ src, int n, int w, int lane,
+                                           uint16_t* cnt, int n_buckets, int* status) {
+  for (int st = 0; st < kWarpKeys / 32; ++st) {
+    const int i = w * kWarpKeys + st * 32 + lane;
+    uint32_t b = 0xffffffffu;
+    if (i < n) {
+      b = (uint32_t)src[i];
+      if (b >= (uint32_t)n_buckets) {
+        if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
+        b = (uint32_t)n_buckets - 1;
+      }
+    }
+    const uint32_t peers = __match_any_sync(0xffffffffu, b);
+    const int leader = __ffs(peers) - 1;
+    if (i < n && lane == leader) cnt[b] = (uint16_t)(cnt[b] + __popc(peers));
+    __syncwarp();
+  }
+}
+
+__global__ void __launch_bounds__(kWarpsPerTile * 32)
+warp_count_kernel(const int32_t* __restrict__ bucket, int32_t* __restrict__ counts, int L,
+                  int n_buckets, int tiles, int* status) {
+  extern __shared__ uint8_t sm[];
+  uint16_t* hist = reinterpret_cast<uint16_t*>(sm);     // [warps][n_buckets]
+  const int tile = blockIdx.x % tiles;
+  const int64_t seg = blockIdx.x / tiles;
+  const int64_t p0 = (int64_t)tile * kWTile;
+  const int n = min(kWTile, (int)(L - p0));
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kWarpsPerTile * n_buckets; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  warp_count(bucket + seg * L + p0, n, w, lane, hist + w * n_buckets, n_buckets, status);
+  __syncthreads();
+  int32_t* out = counts + seg * n_buckets * (int64_t)tiles + tile;
+  for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
+    int tot = 0;
+#pragma unroll
+    for (int ww = 0; ww < kWarpsPerTile; ++ww) tot += hist[ww * n_buckets + b];
+    out[(int64_t)b * tiles] = tot;
+  }
+}
+
+__global__ void __launch_bounds__(kWarpsPerTile * 32)
+warp_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restrict__ counts,
+                    const int32_t* __restrict__ base, int32_t* __restrict__ perm, int L,
+                    int n_buckets, int tiles) {
+  extern __shared__ uint8_t sm[];
+  uint16_t* cnt = reinterpret_cast<uint16_t*>(sm);      // [warps][n_buckets]
+  int32_t* off = reinterpret_cast<int32_t*>(sm + (size_t)kWarpsPerTile * n_buckets * 2);
+  const int tile = blockIdx.x % tiles;
+  const int64_t seg = blockIdx.x / tiles;
+  const int64_t p0 = (int64_t)tile * kWTile;
+  const int n = min(kWTile, (int)(L - p0));
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t* src = bucket + seg * L + p0;
+  for (int i = threadIdx.x; i < kWarpsPerTile * n_buckets; i += blockDim.x) cnt[i] = 0;
+  for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
+    const int64_t row = seg * n_buckets + b;
+    off[b] = base[row] + counts[row * tiles + tile];
+  }
+  __syncthreads();
+  warp_count(src, n, w, lane, cnt + w * n_buckets, n_buckets, nullptr);
+  __syncthreads();
+  // exclusive prefix over warps: cnt[w][b] becomes the start of warp w's run
+  for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
+    int acc = 0;
+#pragma unroll
+    for (int ww = 0; ww < kWarpsPerTile; ++ww) {
+      const int c = cnt[ww * n_buckets + b];
+      cnt[ww * n_buckets + b] = (uint16_t)acc;
+      acc += c;
+    }
+  }
+  __syncthreads();
+  uint16_t* mine = cnt + w * n_buckets;
+  int32_t* out = perm + seg * L;
+  for (int st = 0; st < kWarpKeys / 32; ++st) {
+    const int i = w * kWarpKeys + st * 32 + lane;
+    uint32_t b = 0xffffffffu;
+    if (i < n) {
+      b = (uint32_t)src[i];
+      if (b >= (uint32_t)n_buckets) b = (uint32_t)n_buckets - 1;
+    }
+    const uint32_t peers = __match_any_sync(0xffffffffu, b);
+    const int leader = __ffs(peers) - 1;
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (i < n) out[off[b] + mine[b] + rank] = (int32_t)(p0 + i);
+    __syncwarp();
+    if (i < n && lane == leader) mine[b] = (uint16_t)(mine[b] + __popc(peers));
+    __syncwarp();
+  }
+}
+
+bool warp_path(const lsh_problem& p) { return p.n_buckets <= kWarpMaxBuckets; }
+
 }  // namespace
 
 size_t sort_ws_bytes(const lsh_problem& p) {
   const int64_t S = (int64_t)p.B * p.H * p.n_rounds;
-  const int64_t tiles = (p.L + kTile - 1) / kTile;
-  size_t b = align_up((size_t)S * p.L * 4, 256);
+  const int64_t tiles = warp_path(p) ? (p.L + kWTile - 1) / kWTile : (p.L + kTile - 1) / kTile;
+  size_t b = warp_path(p) ? 0 : align_up((size_t)S * p.L * 4, 256);
   b += align_up((size_t)S * p.n_buckets * tiles * 4, 256);
   b += align_up((size_t)S * p.n_buckets * 4, 256);
   return b;
@@ -187,11 +297,11 @@ size_t sort_ws_bytes(const lsh_problem& p) {
 
 SortWs sort_ws_carve(const lsh_problem& p, void* ws) {
   const int64_t S = (int64_t)p.B * p.H * p.n_rounds;
-  const int64_t tiles = (p.L + kTile - 1) / kTile;
+  const int64_t tiles = warp_path(p) ? (p.L + kWTile - 1) / kWTile : (p.L + kTile - 1) / kTile;
   char* c = (char*)ws;
   SortWs w;
-  w.sorted = (uint32_t*)c;
-  c += align_up((size_t)S * p.L * 4, 256);
+  w.sorted = warp_path(p) ? nullptr : (uint32_t*)c;
+  if (!warp_path(p)) c += align_up((size_t)S * p.L * 4, 256);
   w.counts = (int32_t*)c;
   c += align_up((size_t)S * p.n_buckets * tiles * 4, 256);
   w.base = (int32_t*)c;
@@ -201,8 +311,26 @@ SortWs sort_ws_carve(const lsh_problem& p, void* ws) {
 cudaError_t launch_sort(const lsh_problem& p, const int32_t* bucket, int32_t* perm,
                         const SortWs& ws, int* status, cudaStream_t s) {
   const int64_t S = (int64_t)p.B * p.H * p.n_rounds;
-  const int tiles = (p.L + kTile - 1) / kTile;
   const int64_t rows = S * p.n_buckets;
+  if (warp_path(p)) {
+    const int tiles = (p.L + kWTile - 1) / kWTile;
+    const size_t sm = (size_t)kWarpsPerTile * p.n_buckets * 2 + (size_t)p.n_buckets * 4;
+    cudaError_t e = cudaFuncSetAttribute(warp_count_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWarpSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(warp_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kWarpSmem);
+    if (e != cudaSuccess) return e;
+    warp_count_kernel<<<(unsigned)(S * tiles), kWarpsPerTile * 32, sm, s>>>(bucket, ws.counts, p.L,
+                                                                            p.n_buckets, tiles, status);
+    row_scan_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(ws.counts, ws.base, rows, tiles);
+    bucket_scan_kernel<<<(unsigned)S, 1024, 0, s>>>(ws.base, p.n_buckets);
+    warp_scatter_kernel<<<(unsigned)(S * tiles), kWarpsPerTile * 32, sm, s>>>(
+        bucket, ws.counts, ws.base, perm, p.L, p.n_buckets, tiles);
+    note_launch(4);
+    return cudaGetLastError();
+  }
+  const int tiles = (p.L + kTile - 1) / kTile;
   cudaError_t e = cudaMemsetAsync(ws.counts, 0, (size_t)rows * tiles * 4, s);
   if (e != cudaSuccess) return e;
   tile_sort_kernel<<<(unsigned)(S * tiles), kTileThreads, 0, s>>>(bucket, ws.sorted, ws.counts, p.L,

@@ -109,7 +109,7 @@ def test_workspace_sizes_grow_with_problem():
     _ensure_built()
     L = _lib.lib()
     a = _p()
-    b = _p(L=512)
+    b = _p(L=8192)   # spans several sort tiles
     for f in (L.lsh_sort_workspace_size, L.lsh_fwd_workspace_size, L.lsh_bwd_workspace_size):
         assert 0 < f(ctypes.byref(a)) < f(ctypes.byref(b))
         assert f(ctypes.byref(a)) % 256 == 0
