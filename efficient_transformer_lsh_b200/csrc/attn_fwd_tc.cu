@@ -22,11 +22,11 @@
 //                (exact for |values| < 65504); x stays bf16, whose products
 //                are exact in the Q K^T MMA too. Software-pipelined one job
 //                deep, with the next job's perm entries loaded a job ahead;
-//   warp 4     : TMEM allocation; one thread issues S = Q K^T (three
+//   warp 12    : TMEM allocation; one thread issues S = Q K^T (three
 //                128x64x64 MMAs per pair into a double-buffered TMEM S) and
 //                O = P V with P read from TMEM (A operand) and V from shared
 //                memory (MN-major B operand);
-//   warps 5-8  : softmax warpgroup for even jobs, warps 9-12 for odd jobs —
+//   warps 4-7  : softmax warpgroup for even jobs, warps 8-11 for odd jobs —
 //                one query row per thread, two passes over its S row in TMEM:
 //                (1) causal/self mask and row max, masked values written back;
 //                (2) exp2, row sum, P packed as fp16 pairs into TMEM over S.
@@ -54,7 +54,12 @@ constexpr int kPre = 3;           // side buffers for a unit's previous chunk
 constexpr int kTile = 64 * 128;   // one chunk of 64 rows x 64 16-bit values = 8 KB
 constexpr int kSlotBytes = 4 * kTile;   // x_even | x_odd | v_even | v_odd
 constexpr int kPreBytes = 2 * kTile;    // x_prev | v_prev
-constexpr int kThreads = 416;
+constexpr int kThreads = 512;           // 4 warpgroups
+// Register split (setmaxnreg): launched at 128 per thread (65536 / 512);
+// producers and the MMA warpgroup drop to 56, the two softmax warpgroups
+// rise to 200: 2*128*56 + 2*128*200 = 65536.
+constexpr int kRegsLow = 64, kRegsHigh = 192;
+static_assert(2 * 128 * kRegsLow + 2 * 128 * kRegsHigh <= kThreads * 128, "register split");
 constexpr uint32_t kSCols = 192;        // TMEM columns of one S / P buffer
 constexpr uint32_t kOCol = 2 * kSCols;  // first TMEM column of the O buffers
 
@@ -173,7 +178,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
     bar->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 12) {
     tmem_alloc(&bar->tmem_base, 512);
     tmem_relinquish();
   }
@@ -181,9 +186,11 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
+  const int wgi = warp >> 2;
 
-  if (warp < 4) {
+  if (wgi == 0) {
     // ------------------------------------------------ producers
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
     const int t = threadIdx.x, row = t >> 1, half = t & 1;
     JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
     Job cur, nxt;
@@ -273,9 +280,10 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
     }
     cp_async_wait<0>();
     if (pend && ok) publish();
-  } else if (warp == 4) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
+  } else if (wgi == 3) {
+    // ------------------------------------------------ MMA issuer (warp 12)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+    if (warp == 12 && lane == 0) {
       const uint32_t idesc_s = idesc_f16(128, 64, 1, false, false);   // Q K^T: bf16, K-major
       const uint32_t idesc_o = idesc_f16(128, 64, 0, false, true);    // P V, V MN-major
       const uint32_t slots_a = smem_u32(slots), pres_a = smem_u32(pres);
@@ -358,7 +366,8 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
     }
   } else {
     // ------------------------------------------------ softmax warpgroups
-    const int wg = (warp - 5) >> 2;             // 0: even jobs, 1: odd jobs
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+    const int wg = wgi - 1;                     // 0: even jobs, 1: odd jobs
     const int q = warp & 3;                     // TMEM lane quarter (rows 32q..32q+31)
     const int row = q * 32 + lane;              // query row in the pair tile
     const bool odd_row = row >= 64;             // row belongs to chunk 2p+1
@@ -422,18 +431,20 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
       const int* kp_hi = kb0 == 0 ? bar->kpos[s] : bar->kpos[s] + 64;
       const bool lo_ok = kb0 == 0 ? has_prev : true;
       // pass 1: mask and row max over this row's 128 keys; masked values
-      // (-inf) are written back so pass 2 needs no positions
-      float mx = -INFINITY;
+      // (-inf) are written back so pass 2 needs no positions. Two TMEM loads
+      // per wait and four independent max chains keep latency off the path.
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        const uint32_t col = (uint32_t)(kb0 * 64 + c4 * 32);
-        uint32_t sv[32];
-        tmem_ld32(sbuf + col, sv);
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const uint32_t col = (uint32_t)(kb0 * 64 + c2 * 64);
+        uint32_t sv[64];
+        tmem_ld32(sbuf + col, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(sbuf + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
         tmem_ld_wait();
-        const int* kp = (c4 < 2) ? kp_lo + c4 * 32 : kp_hi + (c4 - 2) * 32;
-        const bool blk_ok = (c4 < 2) ? lo_ok : true;
+        const int* kp = (c2 == 0) ? kp_lo : kp_hi;
+        const bool blk_ok = (c2 == 0) ? lo_ok : true;
 #pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
+        for (int i4 = 0; i4 < 16; ++i4) {
           const int4 k4 = blk_ok ? *reinterpret_cast<const int4*>(kp + 4 * i4)
                                  : make_int4(0, 0, 0, 0);
           const int kk[4] = {k4.x, k4.y, k4.z, k4.w};
@@ -443,32 +454,38 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
             const bool valid = blk_ok && (kCausal ? (kk[e] < qpos) : (kk[e] != qpos));
             const float x = valid ? __uint_as_float(sv[i]) : -INFINITY;
             sv[i] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
+            mx4[e] = fmaxf(mx4[e], x);
           }
         }
-        tmem_st32(sbuf + col, sv);
+        tmem_st32(sbuf + col, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_st32(sbuf + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       }
       tmem_st_wait();
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       const bool has = mx != -INFINITY;
       const float neg = has ? -mx * scale_log2 : 0.f;
       // pass 2: P = exp2(scale * (s - max)) as fp16 pairs into TMEM over S;
       // P column block kb lives at TMEM columns [32 kb, 32 kb + 32)
-      float l = 0.f;
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t sv[32];
-        tmem_ld32(sbuf + (uint32_t)(kb0 * 64 + c4 * 32), sv);
+      for (int c2 = 0; c2 < 2; ++c2) {
+        uint32_t sv[64];
+        const uint32_t col = (uint32_t)(kb0 * 64 + c2 * 64);
+        tmem_ld32(sbuf + col, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(sbuf + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
         tmem_ld_wait();
-        uint32_t pk[16];
+        uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < 32; ++e) {
           const float e0 = ex2(fmaf(__uint_as_float(sv[2 * e]), scale_log2, neg));
           const float e1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), scale_log2, neg));
-          l += e0 + e1;
+          l4[e & 3] += e0 + e1;
           pk[e] = pack_f16x2(e0, e1);
         }
-        tmem_st16(sbuf + (uint32_t)(kb0 * 32 + c4 * 16), pk);
+        tmem_st16(sbuf + (uint32_t)(kb0 * 32 + c2 * 32), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+        tmem_st16(sbuf + (uint32_t)(kb0 * 32 + c2 * 32 + 16), *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
       }
+      const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
       {
         uint32_t z[32];
 #pragma unroll
@@ -492,7 +509,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
