@@ -9,33 +9,37 @@
 //   dqk_i += scale dS_ij x_j (query side: keys are the queries).
 //
 // Work item: a PAIR of key chunks (2p, 2p+1) of one (batch, head, round)
-// segment — 128 keys. The queries that see them are chunks 2p, 2p+1, 2p+2
-// (chunk c sees chunks c-1 and c), 192 queries in three blocks; key rows of
-// chunk 2p use query blocks 0-1, rows of chunk 2p+1 use blocks 1-2.
-//   S^T  = X_K X_Q^T  and  dP^T = V_K dO_Q^T       (M=128 keys, N=3x64)
-//   P^T, dS^T per key row (one thread per TMEM lane)
-//   dV   = P^T dO_Q   (P^T from TMEM)              (complete for the keys)
-//   dK   = dS^T X_Q   (dS^T from shared memory)    (complete for the keys)
-//   R0   = dS[blocks 0,1] X_K  — the query-side term for chunks 2p, 2p+1,
-//          i.e. for the same tokens as the key rows, lane for lane;
-//   R1   = dS[block 2, zeros] X_K — the query-side term for chunk 2p+2
-//          (its other half comes from the next pair's work item).
-// The dS operands of R0/R1 are the transposed (MN-major) reading of the
-// dS^T tile. Each key row then adds scale*(dK + R0) to dqk and dV to dv with
-// vector atomics (rounds and neighbouring items accumulate there); rows of
-// chunk 2p+2 add scale*R1.
+// segment — 128 keys, one per TMEM lane. The queries that see them are
+// chunks 2p, 2p+1, 2p+2 (chunk c sees chunks c-1 and c): three query blocks
+// of 64; key rows of chunk 2p see blocks 0-1, rows of chunk 2p+1 blocks 1-2.
+// Each block is one pipeline step:
+//   S^T = X_K X_qb^T, dP^T = V_K dO_qb^T        (M=128 keys, N=64)
+//   P^T (fp16, in place over S^T in TMEM) and dS^T (fp16, shared memory)
+//   dV += P^T dO_qb,  dK += dS^T X_qb           (accumulated in TMEM)
+// and after blocks 0-1 / block 2 the query-side terms through the
+// transposed (MN-major) reading of the dS^T tiles:
+//   R0 = dS[blocks 0,1] X_K — for chunks 2p, 2p+1, i.e. the same tokens as
+//        the key rows, lane for lane: accumulated straight into dK;
+//   R1 = dS[block 2, zeros] X_K — for chunk 2p+2, which is the first key
+//        chunk of the next pair: written into the OTHER accumulator set's dK,
+//        so that the next item of the same unit adds its own terms on top.
+//        At the end of a unit it is flushed on its own.
+// Each key row finally adds dV to dv and scale*dK to dqk (rounds and
+// neighbouring items meet there) with vector atomics.
 //
-// Warp roles (persistent CTA, one per SM):
-//   warps 0-3: producers — cp.async gathers of x, dout (3 chunks) and v (2
-//              chunks) into a 2-slot ring, in-place bf16 -> fp16 conversion,
-//              per-query position, log2-scaled LSE and D;
-//   warp 4   : TMEM allocation and the MMA-issuing thread;
-//   warps 5-8 and 9-12: two warpgroups, one thread per key row in each; the
-//              first takes the row's first query block, the second its second
-//              (P and dS are elementwise once LSE and D are known, so the two
-//              halves need no exchange); then the gradient epilogue with
-//              atomics, dV and R1 from the first warpgroup, dK + R0 from the
-//              second.
+// TMEM (512 columns): two S^T|dP^T buffers (steps alternate) and two
+// dV|dK accumulator sets (items alternate), so that the S^T/dP^T products
+// of the next step, the softmax of this one and the flush of the previous
+// item all run at once.
+//
+// Warp roles (persistent CTA, one per SM), register budgets via setmaxnreg:
+//   warps 0-2  : producers — cp.async gathers of x, dout (3 chunks) and v
+//                (2 chunks) into a 2-slot ring, in-place bf16 -> fp16
+//                conversion, per-query position, log2-scaled LSE and D;
+//   warp 3     : TMEM allocation and the MMA-issuing thread;
+//   warps 4-7  : gradient flush of the previous item (one thread per row);
+//   warps 8-11, 12-15: two softmax warpgroups, one per S^T buffer (even and
+//                odd steps), one thread per key row.
 #include <cuda_fp16.h>
 #include <stddef.h>
 
@@ -58,37 +62,38 @@ constexpr int kX = 0, kV = 3 * kTile, kDo = 5 * kTile;
 constexpr int kSlotBytes = 8 * kTile;  // 64 KB
 constexpr int kDsBlock = 128 * 128;    // 128 key rows x 64 query columns
 constexpr int kDsBytes = 4 * kDsBlock; // dS^T blocks 0,1,2 + a zero block
-constexpr int kThreads = 416;
+constexpr int kStageStride = 144;      // bytes per staged half-row (128 + 16 pad)
+constexpr int kStageBytes = 4 * 32 * kStageStride;
+constexpr int kThreads = 512;
+constexpr int kProducers = 96;
+constexpr int kRegsLow = 104, kRegsFlush = 88, kRegsSmx = 144;
+static_assert(128 * (kRegsLow + kRegsFlush) + 256 * kRegsSmx <= kThreads * 128, "register split");
 // TMEM columns
-constexpr uint32_t kColS = 0, kColDp = 192;      // S^T, dP^T
-constexpr uint32_t kColDv = 96, kColDk = 288;    // accumulators in their upper halves
-constexpr uint32_t kColR0 = 384, kColR1 = 448;
-// P^T (fp16 pairs, 3 x 32 columns) lives in the R0/R1 columns while they are
-// idle: written after the previous item's flush, read by the dV MMAs, which
-// run before the R0/R1 MMAs that overwrite it (MMAs complete in issue order).
-// The S^T/dP^T columns are read by both key-row warpgroups, so nothing is
-// written there before both have read them.
-constexpr uint32_t kColP = 384;
+constexpr uint32_t kColBuf = 0;        // + 128 w: S^T (64) | dP^T (64); P^T over S^T
+constexpr uint32_t kColAcc = 256;      // + 128 a: dV (64) | dK (64)
 
 struct __align__(16) BwdBar {
   uint64_t slot_full[kSlots];
   uint64_t slot_free[kSlots];
-  uint64_t s_full;
-  uint64_t p_full;
-  uint64_t g_full;
-  uint64_t g_free;
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t g_full[2];
+  uint64_t acc_free[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
   alignas(16) int qpos[kSlots][192];     // positions of query columns (= key rows for 0..127)
   alignas(16) float lse2[kSlots][192];   // LSE * log2(e); +inf for self-attending rows
   alignas(16) float dval[kSlots][192];   // D = dout . out
+  alignas(16) int tok[4][192];           // positions again, per item (read by the flush)
 };
 static_assert(offsetof(BwdBar, qpos) % 16 == 0 && offsetof(BwdBar, lse2) % 16 == 0 &&
                   offsetof(BwdBar, dval) % 16 == 0,
               "per-column arrays are read with 16-byte loads");
 
-constexpr size_t kSmemBytes = 1024 + kSlots * kSlotBytes + kDsBytes + sizeof(BwdBar);
+constexpr size_t kSmemBytes =
+    1024 + kSlots * kSlotBytes + kDsBytes + kStageBytes + sizeof(BwdBar);
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 struct Job {
   int64_t seg;
@@ -136,6 +141,9 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                "f"(c), "f"(d)
                : "memory");
 }
+// A wait's outcome made uniform across the warp, so that a timeout seen by
+// one lane never leaves the others inside a warp-collective instruction.
+__device__ __forceinline__ bool warp_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 __device__ __forceinline__ void issue_row(const __nv_bfloat16* __restrict__ src_row, uint8_t* tile,
                                           int row, int half) {
@@ -154,31 +162,24 @@ __device__ __forceinline__ void convert_row(uint8_t* tile, int row, int half) {
   }
 }
 
-// Adds scale * (64 consecutive TMEM columns of each lane [+ another 64]) to
-// the 64-float global row `row_of_lane` of that lane (token `tok`, or none
-// when tok < 0). The warp stages its 32 half-rows in shared memory and
-// re-reads them so that each vector atomic instruction covers four whole
-// 128-byte lines (8 lanes per row) instead of 32 scattered 16-byte pieces.
-constexpr int kStageStride = 144;   // bytes per staged half-row (128 + 16 pad)
-__device__ __forceinline__ void flush_rows(float* base, int tok, uint32_t ta, uint32_t tb,
-                                           bool two, float scale, uint8_t* stage, int lane) {
+// Adds scale * (64 consecutive TMEM columns of each lane) to the 64-float
+// global row of that lane's token `tok` (none when tok < 0). The warp stages
+// its 32 half-rows in shared memory and re-reads them so that each vector
+// atomic instruction covers four whole 128-byte lines (8 lanes per row)
+// instead of 32 scattered 16-byte pieces.
+__device__ __forceinline__ void flush_rows(float* base, int tok, uint32_t ta, float scale,
+                                           uint8_t* stage, int lane) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    uint32_t a[32], b[32];
+    uint32_t a[32];
     tmem_ld32(ta + 32 * h, a);
-    if (two) tmem_ld32(tb + 32 * h, b);
     tmem_ld_wait();
     uint8_t* mine = stage + lane * kStageStride;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      float x[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float val = __uint_as_float(a[4 * c + e]);
-        if (two) val += __uint_as_float(b[4 * c + e]);
-        x[e] = val * scale;
-      }
-      *reinterpret_cast<float4*>(mine + 16 * c) = make_float4(x[0], x[1], x[2], x[3]);
+      *reinterpret_cast<float4*>(mine + 16 * c) =
+          make_float4(__uint_as_float(a[4 * c]) * scale, __uint_as_float(a[4 * c + 1]) * scale,
+                      __uint_as_float(a[4 * c + 2]) * scale, __uint_as_float(a[4 * c + 3]) * scale);
     }
     __syncwarp();
     const int piece = lane & 7;
@@ -205,8 +206,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* slots = smem;
   uint8_t* dsb = slots + kSlots * kSlotBytes;
-  static_assert(8 * 32 * kStageStride <= 3 * kDsBlock, "flush staging fits in the dS^T blocks");
-  BwdBar* bar = (BwdBar*)(dsb + kDsBytes);
+  uint8_t* stage_base = dsb + kDsBytes;
+  BwdBar* bar = (BwdBar*)(stage_base + kStageBytes);
   volatile int* abort = &bar->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -215,13 +216,15 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSlots; ++s) {
-      mbar_init(&bar->slot_full[s], 128);
+      mbar_init(&bar->slot_full[s], kProducers);
       mbar_init(&bar->slot_free[s], 1);
     }
-    mbar_init(&bar->s_full, 1);
-    mbar_init(&bar->p_full, 256);
-    mbar_init(&bar->g_full, 1);
-    mbar_init(&bar->g_free, 256);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&bar->s_full[w], 1);
+      mbar_init(&bar->p_full[w], 128);
+      mbar_init(&bar->g_full[w], 1);
+      mbar_init(&bar->acc_free[w], 128);
+    }
     mbar_init(&bar->mma_done, 1);
     bar->abort = 0;
     fence_mbar_init();
@@ -230,7 +233,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
   for (int i = threadIdx.x; i < kDsBlock / 16; i += kThreads)
     reinterpret_cast<uint4*>(dsb + 3 * kDsBlock)[i] = make_uint4(0u, 0u, 0u, 0u);
   fence_proxy_async();
-  if (warp == 4) {
+  if (warp == 3) {
     tmem_alloc(&bar->tmem_base, 512);
     tmem_relinquish();
   }
@@ -238,251 +241,344 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
+  const int wgi = warp >> 2;
 
-  if (warp < 4) {
-    // ------------------------------------------------ producers
-    const int t = threadIdx.x, row = t >> 1, half = t & 1;
-    JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
-    Job j;
-    int n = 0;
-    while (it.next(j)) {
-      const int s = n % kSlots;
-      if (n >= kSlots &&
-          !mbar_wait(&bar->slot_free[s], (uint32_t)(n / kSlots - 1) & 1u, abort, status))
-        break;
-      const int64_t bh = j.seg / n_rounds;
-      const int nc = min(3, n_chunks - 2 * j.p);     // chunks 2p .. 2p+nc-1 exist
-      uint8_t* sl = slots + s * kSlotBytes;
-      const __nv_bfloat16* xb = qk + bh * L * 64;
-      const __nv_bfloat16* vb = v + bh * L * 64;
-      const __nv_bfloat16* gb = dout + bh * L * 64;
-      int pos[3];
-      float l2[3], dd[3];
-#pragma unroll
-      for (int c = 0; c < 3; ++c) {
-        pos[c] = 0;
-        if (c < nc) {
-          int ps = perm[j.seg * L + (int64_t)(2 * j.p + c) * kM + row];
-          if ((unsigned)ps >= (unsigned)L) {
-            if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
-            ps = 0;
-          }
-          pos[c] = ps;
+  if (wgi == 0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+    if (warp < 3) {
+      // ---------------------------------------------- producers: warp c gathers
+      // chunk 2p+c (x, dout, and v for c < 2). Eight lanes cover one 128-byte
+      // row, so each cp.async instruction moves four whole rows.
+      const int c = warp;
+      const int ch = lane & 7, rsub = lane >> 3;
+      JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
+      Job j, jn;
+      bool have = it.next(j);
+      // positions of rows lane and 32+lane of chunk 2p+c, loaded one item ahead
+      auto load_pos = [&](const Job& jj, int& pa, int& pb) {
+        pa = pb = 0;
+        if (c < min(3, n_chunks - 2 * jj.p)) {
+          const int32_t* pj = perm + jj.seg * L + (int64_t)(2 * jj.p + c) * kM;
+          pa = __ldg(pj + lane);
+          pb = __ldg(pj + 32 + lane);
         }
-      }
-#pragma unroll
-      for (int c = 0; c < 3; ++c) {
-        if (c < nc) {
-          issue_row(xb + (int64_t)pos[c] * 64, sl + kX + c * kTile, row, half);
-          issue_row(gb + (int64_t)pos[c] * 64, sl + kDo + c * kTile, row, half);
-          if (c < 2) issue_row(vb + (int64_t)pos[c] * 64, sl + kV + c * kTile, row, half);
+      };
+      int pa = 0, pb = 0;
+      if (have) load_pos(j, pa, pb);
+      int n = 0;
+      while (have) {
+        const bool have_next = it.next(jn);
+        int pa_n = 0, pb_n = 0;
+        if (have_next) load_pos(jn, pa_n, pb_n);
+        const int s = n % kSlots;
+        if (n >= kSlots &&
+            !warp_ok(mbar_wait(&bar->slot_free[s], (uint32_t)(n / kSlots - 1) & 1u, abort, status)))
+          break;
+        const int64_t bh = j.seg / n_rounds;
+        const bool live = c < min(3, n_chunks - 2 * j.p);
+        uint8_t* sl = slots + s * kSlotBytes;
+        if ((unsigned)pa >= (unsigned)L || (unsigned)pb >= (unsigned)L) {
+          if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
+          if ((unsigned)pa >= (unsigned)L) pa = 0;
+          if ((unsigned)pb >= (unsigned)L) pb = 0;
         }
-      }
-      cp_async_commit();
+        if (live) {
+          const __nv_bfloat16* xb = qk + bh * L * 64 + ch * 8;
+          const __nv_bfloat16* gb = dout + bh * L * 64 + ch * 8;
+          const __nv_bfloat16* vb = v + bh * L * 64 + ch * 8;
+          const uint32_t tx = smem_u32(sl + kX + c * kTile), tg = smem_u32(sl + kDo + c * kTile),
+                         tv = smem_u32(sl + kV + c * kTile);
 #pragma unroll
-      for (int c = 0; c < 3; ++c) {
-        l2[c] = 0.f;
-        dd[c] = 0.f;
-        if (c < nc && half == 0) {
-          const float lv = lse[bh * L + pos[c]];
-          l2[c] = (lv == -INFINITY) ? INFINITY : lv * kLog2e;
-          dd[c] = Dg[bh * L + pos[c]];
-        }
-      }
-      cp_async_wait<0>();
-#pragma unroll
-      for (int c = 0; c < 3; ++c) {
-        if (c < nc) {
-          convert_row(sl + kX + c * kTile, row, half);
-          convert_row(sl + kDo + c * kTile, row, half);
-          if (c < 2) convert_row(sl + kV + c * kTile, row, half);
-          if (half == 0) {
-            bar->qpos[s][c * 64 + row] = pos[c];
-            bar->lse2[s][c * 64 + row] = l2[c];
-            bar->dval[s][c * 64 + row] = dd[c];
+          for (int g = 0; g < 16; ++g) {
+            const int row = 4 * g + rsub;
+            const int64_t pos = __shfl_sync(0xffffffffu, g < 8 ? pa : pb, row & 31);
+            const uint32_t off = row * 128 + (((uint32_t)ch ^ (uint32_t)(row & 7)) << 4);
+            cp_async16(tx + off, xb + pos * 64);
+            cp_async16(tg + off, gb + pos * 64);
+            if (c < 2) cp_async16(tv + off, vb + pos * 64);
           }
         }
+        cp_async_commit();
+        // per query column: position, LSE, D (while the rows are in flight)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int q = c * 64 + k * 32 + lane;
+          const int pos = k ? pb : pa;
+          int tp = -1;
+          float l2 = 0.f, dd = 0.f;
+          if (live) {
+            const float lv = lse[bh * L + pos];
+            l2 = (lv == -INFINITY) ? INFINITY : lv * kLog2e;
+            dd = Dg[bh * L + pos];
+            tp = pos;
+          }
+          bar->qpos[s][q] = tp;
+          bar->lse2[s][q] = l2;
+          bar->dval[s][q] = dd;
+          bar->tok[n & 3][q] = tp;
+        }
+        cp_async_wait<0>();
+        if (live) {
+#pragma unroll
+          for (int g = 0; g < 16; ++g) {
+            const int row = 4 * g + rsub;
+            const uint32_t off = row * 128 + (((uint32_t)ch ^ (uint32_t)(row & 7)) << 4);
+            convert_piece_bf16_to_f16(sl + kX + c * kTile + off);
+            convert_piece_bf16_to_f16(sl + kDo + c * kTile + off);
+            if (c < 2) convert_piece_bf16_to_f16(sl + kV + c * kTile + off);
+          }
+        }
+        fence_proxy_async();
+        mbar_arrive(&bar->slot_full[s]);
+        j = jn;
+        pa = pa_n;
+        pb = pb_n;
+        have = have_next;
+        ++n;
       }
-      fence_proxy_async();
-      mbar_arrive(&bar->slot_full[s]);
-      ++n;
-    }
-  } else if (warp == 4) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (lane == 0) {
+      // ---------------------------------------------- MMA issuer
       const uint32_t idesc_kk = idesc_f16(128, 64, 0, false, false);   // both K-major
       const uint32_t idesc_kn = idesc_f16(128, 64, 0, false, true);    // B MN-major
       const uint32_t idesc_nn = idesc_f16(128, 64, 0, true, true);     // A and B MN-major
       const uint32_t slots_a = smem_u32(slots), ds_a = smem_u32(dsb);
+      // descriptor templates (start address 0); a shared-memory address below
+      // 256 KB is added to the 14-bit start-address field as addr >> 4
+      const uint64_t t_k = smem_desc(0, 16, 1024);        // K-major
+      const uint64_t t_n = smem_desc(0, kTile, 1024);     // MN-major input tile
+      const uint64_t t_d = smem_desc(0, kDsBlock, 1024);  // MN-major reading of dS^T
+      auto dsc = [](uint64_t t, uint32_t addr) { return t + (uint64_t)(addr >> 4); };
+      int acc_seen[2] = {0, 0};
+      // waits until the flushes of the first `need` items that used set `a` are done
+      auto wait_acc = [&](int a, int need) -> bool {
+        while (acc_seen[a] < need) {
+          if (!mbar_wait(&bar->acc_free[a], (uint32_t)acc_seen[a] & 1u, abort, status))
+            return false;
+          ++acc_seen[a];
+        }
+        return true;
+      };
+      // S^T and dP^T of step (item nn, query block qb) into buffer (3 nn + qb) & 1
+      auto issue_s = [&](int nn, int qb, int nc, uint32_t sl) {
+        const int w = (3 * nn + qb) & 1;
+        if (qb < nc) {
+          const uint32_t d = tmem + kColBuf + (uint32_t)w * 128;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            mma_ss(d, dsc(t_k, sl + kX + ks * 32),
+                   dsc(t_k, sl + kX + qb * kTile + ks * 32), idesc_kk, ks > 0);
+            mma_ss(d + 64, dsc(t_k, sl + kV + ks * 32),
+                   dsc(t_k, sl + kDo + qb * kTile + ks * 32), idesc_kk, ks > 0);
+          }
+        }
+        mma_commit(&bar->s_full[w]);
+      };
+      auto wait_p = [&](int g) {
+        return mbar_wait(&bar->p_full[g & 1], (uint32_t)(g >> 1) & 1u, abort, status);
+      };
+      // dV += P^T dO_qb ; dK += dS^T_qb X_qb
+      auto issue_g = [&](int g, int qb, uint32_t sl, uint32_t acc, bool acc_v, bool acc_k) {
+        const uint32_t pt = tmem + kColBuf + (uint32_t)(g & 1) * 128;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          mma_ts(acc, pt + ks * 8, dsc(t_n, sl + kDo + qb * kTile + ks * 2048),
+                 idesc_kn, acc_v || ks > 0);
+          mma_ss(acc + 64, dsc(t_k, ds_a + qb * kDsBlock + ks * 32),
+                 dsc(t_n, sl + kX + qb * kTile + ks * 2048), idesc_kn, acc_k || ks > 0);
+        }
+      };
       JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
-      Job j;
+      Job cur, nxt;
+      bool have = it.next(cur);
+      bool ok = true;
+      if (have) {
+        ok = mbar_wait(&bar->slot_full[0], 0u, abort, status);
+        if (ok) {
+          tc_fence_after();
+          const int nc = min(3, n_chunks - 2 * cur.p);
+          issue_s(0, 0, nc, slots_a);
+          issue_s(0, 1, nc, slots_a);
+        }
+      }
       int n = 0;
-      while (it.next(j)) {
-        const int s = n % kSlots;
-        if (!mbar_wait(&bar->slot_full[s], (uint32_t)(n / kSlots) & 1u, abort, status)) break;
-        if (n >= 1 && !mbar_wait(&bar->g_free, (uint32_t)(n - 1) & 1u, abort, status)) break;
-        tc_fence_after();
-        const int nc = min(3, n_chunks - 2 * j.p);
+      bool prev_r1_alone = false;   // the previous item left R1 rows for its own flush
+      while (ok && have) {
+        const bool have_next = it.next(nxt);
+        const int s = n % kSlots, a = n & 1;
+        const int nc = min(3, n_chunks - 2 * cur.p);
         const uint32_t sl = slots_a + s * kSlotBytes;
-        // S^T = X_K X_Q^T and dP^T = V_K dO_Q^T, one N=64 block per query chunk
-#pragma unroll
-        for (int qb = 0; qb < 3; ++qb) {
-          if (qb >= nc) continue;
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            mma_ss(tmem + kColS + qb * 64, smem_desc(sl + kX + ks * 32, 16, 1024),
-                   smem_desc(sl + kX + qb * kTile + ks * 32, 16, 1024), idesc_kk, ks > 0);
-            mma_ss(tmem + kColDp + qb * 64, smem_desc(sl + kV + ks * 32, 16, 1024),
-                   smem_desc(sl + kDo + qb * kTile + ks * 32, 16, 1024), idesc_kk, ks > 0);
-          }
-        }
-        mma_commit(&bar->s_full);
-        if (!mbar_wait(&bar->p_full, (uint32_t)n & 1u, abort, status)) break;
+        const uint32_t acc = tmem + kColAcc + (uint32_t)a * 128;
+        const int g0 = 3 * n;
+        // ---- block 0 (always present)
+        if (!wait_p(g0) || !wait_acc(a, n >> 1)) break;
+        if (prev_r1_alone && !wait_acc(a ^ 1, ((n - 1) >> 1) + 1)) break;
         tc_fence_after();
-        bool acc_v = false, acc_k = false;
-#pragma unroll
-        for (int qb = 0; qb < 3; ++qb) {
-          if (qb >= nc) continue;
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            // dV += P^T (TMEM) . dO_Q ; dK += dS^T (smem, K-major) . X_Q
-            mma_ts(tmem + kColDv, tmem + kColP + qb * 32 + ks * 8,
-                   smem_desc(sl + kDo + qb * kTile + ks * 2048, 8192, 1024), idesc_kn, acc_v);
-            acc_v = true;
-            mma_ss(tmem + kColDk, smem_desc(ds_a + qb * kDsBlock + ks * 32, 16, 1024),
-                   smem_desc(sl + kX + qb * kTile + ks * 2048, 8192, 1024), idesc_kn, acc_k);
-            acc_k = true;
-          }
-        }
-        // query-side terms through the transposed reading of dS^T
+        issue_g(g0, 0, sl, acc, false, !cur.first);
+        issue_s(n, 2, nc, sl);
+        // ---- block 1, then R0 = dS[blocks 0,1] X_K into dK
+        if (!wait_p(g0 + 1)) break;
+        tc_fence_after();
+        if (nc > 1) issue_g(g0 + 1, 1, sl, acc, true, true);
         const int kkeys = nc >= 2 ? 8 : 4;       // K = keys present (16 per step)
-        for (int ks = 0; ks < kkeys; ++ks) {
-          mma_ss(tmem + kColR0, smem_desc(ds_a + ks * 2048, kDsBlock, 1024),
-                 smem_desc(sl + kX + ks * 2048, 8192, 1024), idesc_nn, ks > 0);
-          if (nc == 3)
-            mma_ss(tmem + kColR1, smem_desc(ds_a + 2 * kDsBlock + ks * 2048, kDsBlock, 1024),
-                   smem_desc(sl + kX + ks * 2048, 8192, 1024), idesc_nn, ks > 0);
+        for (int ks = 0; ks < kkeys; ++ks)
+          mma_ss(acc + 64, dsc(t_d, ds_a + ks * 2048),
+                 dsc(t_n, sl + kX + ks * 2048), idesc_nn, true);
+        int nc_next = 0;
+        uint32_t sl_next = 0;
+        if (have_next) {
+          const int sn = (n + 1) % kSlots;
+          if (!mbar_wait(&bar->slot_full[sn], (uint32_t)((n + 1) / kSlots) & 1u, abort, status))
+            break;
+          tc_fence_after();
+          nc_next = min(3, n_chunks - 2 * nxt.p);
+          sl_next = slots_a + sn * kSlotBytes;
+          issue_s(n + 1, 0, nc_next, sl_next);
         }
-        mma_commit(&bar->g_full);
+        // ---- block 2, then R1 = dS[block 2, zeros] X_K into the other set's dK
+        if (!wait_p(g0 + 2)) break;
+        tc_fence_after();
+        if (nc == 3) {
+          issue_g(g0 + 2, 2, sl, acc, true, true);
+          if (!wait_acc(a ^ 1, (n + 1) >> 1)) break;
+          tc_fence_after();
+          const uint32_t acc2 = tmem + kColAcc + (uint32_t)(a ^ 1) * 128;
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ss(acc2 + 64, dsc(t_d, ds_a + 2 * kDsBlock + ks * 2048),
+                   dsc(t_n, sl + kX + ks * 2048), idesc_nn, ks > 0);
+        }
+        mma_commit(&bar->g_full[a]);
         mma_commit(&bar->slot_free[s]);
+        prev_r1_alone = cur.last && nc == 3;
+        if (have_next) issue_s(n + 1, 1, nc_next, sl_next);
+        cur = nxt;
+        have = have_next;
         ++n;
       }
       mma_commit(&bar->mma_done);
       int dummy = 0;
       mbar_wait(&bar->mma_done, 0, (volatile int*)&dummy, status);
     }
-  } else {
-    // ------------------------------------------------ key rows: P, dS, gradients
-    const int kwg = (warp - 5) >> 2;           // 0: first query block, 1: second
+  } else if (wgi == 1) {
+    // ------------------------------------------------ gradient flush
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsFlush));
     const int q = warp & 3;
-    const int row = q * 32 + lane;             // key row = TMEM lane
-    const bool odd_row = row >= 64;
-    const int qb0 = odd_row ? 1 : 0;           // first query block of this key row
-    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const uint32_t tl = tmem + lane_off;
+    const int row = q * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+    uint8_t* stage = stage_base + q * (32 * kStageStride);
     JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
     Job j;
     int n = 0;
     while (it.next(j)) {
-      const int s = n % kSlots;
-      if (!mbar_wait(&bar->s_full, (uint32_t)n & 1u, abort, status)) break;
+      const int a = n & 1;
+      if (!warp_ok(mbar_wait(&bar->g_full[a], (uint32_t)(n >> 1) & 1u, abort, status))) break;
       tc_fence_after();
       const int nc = min(3, n_chunks - 2 * j.p);
-      const bool row_live = row < 64 * min(nc, 2);
-      const int kpos = bar->qpos[s][row];
-      // position of this lane's row of chunk 2p+2 (read now: the slot may be
-      // refilled once the gradient MMAs are done)
-      const int qpos2 = (nc == 3 && !odd_row) ? bar->qpos[s][128 + row] : 0;
-      const int* qp_all = bar->qpos[s];
-      const float* l2_all = bar->lse2[s];
-      const float* d_all = bar->dval[s];
-      {
-        const int qb = qb0 + kwg;
-        const bool blk_ok = qb < nc && row_live;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int col0 = qb * 64 + h * 32;
-          uint32_t sv[32], pv[32];
-          tmem_ld32(tl + kColS + col0, sv);
-          tmem_ld32(tl + kColDp + col0, pv);
-          tmem_ld_wait();
-          uint32_t pk[16], dk[16];
-#pragma unroll
-          for (int i4 = 0; i4 < 8; ++i4) {
-            int4 q4 = make_int4(0, 0, 0, 0);
-            float4 l4 = make_float4(0.f, 0.f, 0.f, 0.f), d4 = l4;
-            if (blk_ok) {
-              q4 = *reinterpret_cast<const int4*>(qp_all + col0 + 4 * i4);
-              l4 = *reinterpret_cast<const float4*>(l2_all + col0 + 4 * i4);
-              d4 = *reinterpret_cast<const float4*>(d_all + col0 + 4 * i4);
-            }
-            const int qq[4] = {q4.x, q4.y, q4.z, q4.w};
-            const float ll[4] = {l4.x, l4.y, l4.z, l4.w};
-            const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
-            float pe[4], de[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int i = 4 * i4 + e;
-              const bool valid = blk_ok && (kCausal ? (kpos < qq[e]) : (kpos != qq[e]));
-              const float pr = ex2(fmaf(__uint_as_float(sv[i]), scale_log2, -ll[e]));
-              pe[e] = valid ? pr : 0.f;
-              de[e] = valid ? pr * (__uint_as_float(pv[i]) - dd[e]) : 0.f;
-            }
-            pk[2 * i4] = pack_f16x2(pe[0], pe[1]);
-            pk[2 * i4 + 1] = pack_f16x2(pe[2], pe[3]);
-            dk[2 * i4] = pack_f16x2(de[0], de[1]);
-            dk[2 * i4 + 1] = pack_f16x2(de[2], de[3]);
-          }
-          // P^T into TMEM (block qb at columns kColP + 32 qb), dS^T into smem
-          tmem_st16(tl + kColP + (uint32_t)(qb * 32 + h * 16), pk);
-          uint8_t* drow = dsb + qb * kDsBlock + row * 128;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int ch = h * 4 + c;
-            *reinterpret_cast<uint4*>(drow + ((ch ^ (row & 7)) << 4)) =
-                make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
-          }
-        }
-      }
-      if (kwg == 1) {
-        // the query block this key row does not see: P = 0 and dS = 0
-        const int zb = odd_row ? 0 : 2;
-        uint32_t z[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) z[e] = 0u;
-        tmem_st32(tl + kColP + (uint32_t)(zb * 32), z);
-        uint8_t* drow = dsb + zb * kDsBlock + row * 128;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          *reinterpret_cast<uint4*>(drow + ((ch ^ (row & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
-      }
-      tmem_st_wait();
-      fence_proxy_async();
-      tc_fence_before();
-      mbar_arrive(&bar->p_full);
-      // gradients of this pair
-      if (!mbar_wait(&bar->g_full, (uint32_t)n & 1u, abort, status)) break;
-      tc_fence_after();
       const int64_t bh = j.seg / n_rounds;
-      // staging: the dS^T blocks are idle until the next item's softmax,
-      // which starts only after every row here has been flushed
-      uint8_t* stage = dsb + (warp - 5) * (32 * kStageStride);
-      const int tok = row_live ? kpos : -1;
-      if (kwg == 0) flush_rows(dv + bh * L * 64, tok, tl + kColDv, 0, false, 1.f, stage, lane);
-      if (kwg == 1)
-        flush_rows(dqk + bh * L * 64, tok, tl + kColDk, tl + kColR0, true, scale, stage, lane);
-      if (kwg == 0 && nc == 3 && !odd_row) {
-        // query-side term of chunk 2p+2 (lanes 0..63 of R1)
-        flush_rows(dqk + bh * L * 64, qpos2, tl + kColR1, 0, false, scale, stage, lane);
+      const int* tk = bar->tok[n & 3];
+      const int tok = row < 64 * min(nc, 2) ? tk[row] : -1;
+      const uint32_t acc = tl + kColAcc + (uint32_t)a * 128;
+      flush_rows(dv + bh * L * 64, tok, acc, 1.f, stage, lane);
+      flush_rows(dqk + bh * L * 64, tok, acc + 64, scale, stage, lane);
+      if (j.last && nc == 3 && q < 2) {
+        // R1 rows (chunk 2p+2) that no later item of this unit picks up
+        flush_rows(dqk + bh * L * 64, tk[128 + row], tl + kColAcc + (uint32_t)(a ^ 1) * 128 + 64,
+                   scale, stage, lane);
       }
       tc_fence_before();
-      mbar_arrive(&bar->g_free);
+      mbar_arrive(&bar->acc_free[a]);
+      ++n;
+    }
+  } else {
+    // ------------------------------------------------ softmax: P^T and dS^T
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSmx));
+    const int w = wgi - 2;                     // S^T buffer = parity of the step
+    const int q = warp & 3;
+    const int row = q * 32 + lane;             // key row = TMEM lane
+    const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + kColBuf + (uint32_t)w * 128;
+    JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
+    Job j;
+    int n = 0, k = 0;
+    bool ok = true;
+    while (ok && it.next(j)) {
+      const int s = n % kSlots;
+      const int nc = min(3, n_chunks - 2 * j.p);
+      for (int qb = 0; qb < 3; ++qb) {
+        if (((3 * n + qb) & 1) != w) continue;
+        if (!warp_ok(mbar_wait(&bar->s_full[w], (uint32_t)k & 1u, abort, status))) {
+          ok = false;
+          break;
+        }
+        ++k;
+        tc_fence_after();
+        if (qb < nc) {
+          const bool active = qb == 1 || (qb == 0 ? row < 64 : row >= 64);
+          uint8_t* drow = dsb + qb * kDsBlock + row * 128;
+          if (active) {
+            const int kpos = bar->qpos[s][row];  // this key row's position
+            const int* qp_all = bar->qpos[s];
+            const float* l2_all = bar->lse2[s];
+            const float* d_all = bar->dval[s];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int col0 = qb * 64 + h * 32;
+              uint32_t sv[32], pv[32];
+              tmem_ld32(tb + h * 32, sv);
+              tmem_ld32(tb + 64 + h * 32, pv);
+              tmem_ld_wait();
+              uint32_t pk[16], dk[16];
+#pragma unroll
+              for (int i4 = 0; i4 < 8; ++i4) {
+                const int4 q4 = *reinterpret_cast<const int4*>(qp_all + col0 + 4 * i4);
+                const float4 l4 = *reinterpret_cast<const float4*>(l2_all + col0 + 4 * i4);
+                const float4 d4 = *reinterpret_cast<const float4*>(d_all + col0 + 4 * i4);
+                const int qq[4] = {q4.x, q4.y, q4.z, q4.w};
+                const float ll[4] = {l4.x, l4.y, l4.z, l4.w};
+                const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+                float pe[4], de[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int i = 4 * i4 + e;
+                  const bool valid = kCausal ? (kpos < qq[e]) : (kpos != qq[e]);
+                  const float pr = ex2(fmaf(__uint_as_float(sv[i]), scale_log2, -ll[e]));
+                  pe[e] = valid ? pr : 0.f;
+                  de[e] = valid ? pr * (__uint_as_float(pv[i]) - dd[e]) : 0.f;
+                }
+                pk[2 * i4] = pack_f16x2(pe[0], pe[1]);
+                pk[2 * i4 + 1] = pack_f16x2(pe[2], pe[3]);
+                dk[2 * i4] = pack_f16x2(de[0], de[1]);
+                dk[2 * i4 + 1] = pack_f16x2(de[2], de[3]);
+              }
+              // P^T over the S^T columns already read; dS^T into shared memory
+              tmem_st16(tb + h * 16, pk);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const int ch = h * 4 + c;
+                *reinterpret_cast<uint4*>(drow + ((ch ^ (row & 7)) << 4)) =
+                    make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
+              }
+            }
+          } else {
+            // a key row that this query block does not see: P = 0 and dS = 0
+            uint32_t z[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) z[e] = 0u;
+            tmem_st32(tb, z);
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+              *reinterpret_cast<uint4*>(drow + ((ch ^ (row & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          tmem_st_wait();
+          fence_proxy_async();
+        }
+        tc_fence_before();
+        mbar_arrive(&bar->p_full[w]);
+      }
       ++n;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 3) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
