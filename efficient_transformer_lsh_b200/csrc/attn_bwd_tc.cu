@@ -14,8 +14,9 @@
 // of 64; key rows of chunk 2p see blocks 0-1, rows of chunk 2p+1 blocks 1-2.
 // Each block is one pipeline step:
 //   S^T = X_K X_qb^T, dP^T = V_K dO_qb^T        (M=128 keys, N=64)
-//   P^T (fp16, in place over S^T in TMEM) and dS^T (fp16, shared memory)
-//   dV += P^T dO_qb,  dK += dS^T X_qb           (accumulated in TMEM)
+//   P^T and dS^T (fp16, in place over S^T and dP^T in TMEM; dS^T also to
+//   shared memory for the query-side products)
+//   dV += P^T dO_qb,  dK += dS^T X_qb           (A from TMEM, accumulated in TMEM)
 // and after blocks 0-1 / block 2 the query-side terms through the
 // transposed (MN-major) reading of the dS^T tiles:
 //   R0 = dS[blocks 0,1] X_K — for chunks 2p, 2p+1, i.e. the same tokens as
@@ -24,8 +25,12 @@
 //        chunk of the next pair: written into the OTHER accumulator set's dK,
 //        so that the next item of the same unit adds its own terms on top.
 //        At the end of a unit it is flushed on its own.
-// Each key row finally adds dV to dv and scale*dK to dqk (rounds and
-// neighbouring items meet there) with vector atomics.
+// The finished rows dV and scale*dK of an item are stored, converted to fp16,
+// as per-round partial gradients in sorted (slot) order — 128 consecutive
+// rows, two TMA tile stores per tensor; unit-end R1 rows go to a small edge
+// buffer. A second kernel then sums, for every token, its rows of all rounds
+// (located through the inverse permutation) into dqk and dv, so no atomics
+// are needed anywhere.
 //
 // TMEM (512 columns): two S^T|dP^T buffers (steps alternate) and two
 // dV|dK accumulator sets (items alternate), so that the S^T/dP^T products
@@ -37,7 +42,8 @@
 //                (2 chunks) into a 2-slot ring, in-place bf16 -> fp16
 //                conversion, per-query position, log2-scaled LSE and D;
 //   warp 3     : TMEM allocation and the MMA-issuing thread;
-//   warps 4-7  : gradient flush of the previous item (one thread per row);
+//   warps 4-7  : gradient flush of the previous item (one thread per row,
+//                fp16 staging in shared memory, TMA stores);
 //   warps 8-11, 12-15: two softmax warpgroups, one per S^T buffer (even and
 //                odd steps), one thread per key row.
 #include <cuda_fp16.h>
@@ -62,8 +68,7 @@ constexpr int kX = 0, kV = 3 * kTile, kDo = 5 * kTile;
 constexpr int kSlotBytes = 8 * kTile;  // 64 KB
 constexpr int kDsBlock = 128 * 128;    // 128 key rows x 64 query columns
 constexpr int kDsBytes = 4 * kDsBlock; // dS^T blocks 0,1,2 + a zero block
-constexpr int kStageStride = 144;      // bytes per staged half-row (128 + 16 pad)
-constexpr int kStageBytes = 4 * 32 * kStageStride;
+constexpr int kStageBytes = 128 * 128; // 128 fp16 rows, 128-byte swizzle
 constexpr int kThreads = 512;
 constexpr int kProducers = 96;
 constexpr int kRegsLow = 104, kRegsFlush = 88, kRegsSmx = 144;
@@ -136,11 +141,6 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
 // A wait's outcome made uniform across the warp, so that a timeout seen by
 // one lane never leaves the others inside a warp-collective instruction.
 __device__ __forceinline__ bool warp_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
@@ -162,35 +162,42 @@ __device__ __forceinline__ void convert_row(uint8_t* tile, int row, int half) {
   }
 }
 
-// Adds scale * (64 consecutive TMEM columns of each lane) to the 64-float
-// global row of that lane's token `tok` (none when tok < 0). The warp stages
-// its 32 half-rows in shared memory and re-reads them so that each vector
-// atomic instruction covers four whole 128-byte lines (8 lanes per row)
-// instead of 32 scattered 16-byte pieces.
-__device__ __forceinline__ void flush_rows(float* base, int tok, uint32_t ta, float scale,
-                                           uint8_t* stage, int lane) {
+// A wait's outcome made uniform across the `n` threads of named barrier `id`
+// (all of them must call it).
+__device__ __forceinline__ bool group_ok(int id, int n, bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "barrier.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)ok), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Converts 64 fp32 TMEM columns of this thread's lane, times `sc`, to fp16
+// and writes them as row `row` of a 128-byte-swizzled staging tile.
+__device__ __forceinline__ void stage_row(uint32_t ta, float sc, uint8_t* stage, int row) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     uint32_t a[32];
     tmem_ld32(ta + 32 * h, a);
     tmem_ld_wait();
-    uint8_t* mine = stage + lane * kStageStride;
+    uint32_t pk[16];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      *reinterpret_cast<float4*>(mine + 16 * c) =
-          make_float4(__uint_as_float(a[4 * c]) * scale, __uint_as_float(a[4 * c + 1]) * scale,
-                      __uint_as_float(a[4 * c + 2]) * scale, __uint_as_float(a[4 * c + 3]) * scale);
-    }
-    __syncwarp();
-    const int piece = lane & 7;
+    for (int i = 0; i < 16; ++i)
+      pk[i] = pack_f16x2(__uint_as_float(a[2 * i]) * sc, __uint_as_float(a[2 * i + 1]) * sc);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int r = 4 * k + (lane >> 3);
-      const int rt = __shfl_sync(0xffffffffu, tok, r);
-      const float4 val = *reinterpret_cast<const float4*>(stage + r * kStageStride + 16 * piece);
-      if (rt >= 0) red_add_v4(base + (int64_t)rt * 64 + 32 * h + 4 * piece, val.x, val.y, val.z, val.w);
+    for (int c = 0; c < 4; ++c) {
+      const int ch = h * 4 + c;
+      *reinterpret_cast<uint4*>(stage + row * 128 + ((ch ^ (row & 7)) << 4)) =
+          make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
     }
-    __syncwarp();
   }
 }
 
@@ -199,7 +206,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __restrict__ v,
                    const __nv_bfloat16* __restrict__ dout, const int32_t* __restrict__ perm,
                    const float* __restrict__ lse, const float* __restrict__ Dg,
-                   float* __restrict__ dqk, float* __restrict__ dv, int L, int n_rounds,
+                   const __grid_constant__ CUtensorMap map_dv,
+                   const __grid_constant__ CUtensorMap map_dqk,
+                   const __grid_constant__ CUtensorMap map_edge, int L, int n_rounds,
                    float scale, float scale_log2, int n_units, int units_per_seg,
                    int* status) {
   extern __shared__ uint8_t smem_raw[];
@@ -376,15 +385,15 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
       auto wait_p = [&](int g) {
         return mbar_wait(&bar->p_full[g & 1], (uint32_t)(g >> 1) & 1u, abort, status);
       };
-      // dV += P^T dO_qb ; dK += dS^T_qb X_qb
+      // dV += P^T dO_qb ; dK += dS^T_qb X_qb (P^T and dS^T from TMEM)
       auto issue_g = [&](int g, int qb, uint32_t sl, uint32_t acc, bool acc_v, bool acc_k) {
         const uint32_t pt = tmem + kColBuf + (uint32_t)(g & 1) * 128;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           mma_ts(acc, pt + ks * 8, dsc(t_n, sl + kDo + qb * kTile + ks * 2048),
                  idesc_kn, acc_v || ks > 0);
-          mma_ss(acc + 64, dsc(t_k, ds_a + qb * kDsBlock + ks * 32),
-                 dsc(t_n, sl + kX + qb * kTile + ks * 2048), idesc_kn, acc_k || ks > 0);
+          mma_ts(acc + 64, pt + 64 + ks * 8, dsc(t_n, sl + kX + qb * kTile + ks * 2048),
+                 idesc_kn, acc_k || ks > 0);
         }
       };
       JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
@@ -464,30 +473,50 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
-    uint8_t* stage = stage_base + q * (32 * kStageStride);
+    const bool issuer = threadIdx.x == 128;
     JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
     Job j;
     int n = 0;
+    // stage -> TMA store of rows [0, 64 nh) to (0, y) of `map`
+    auto store_rows = [&](const CUtensorMap* map, int y, int nh) {
+      fence_proxy_async();
+      named_sync(2, 128);
+      if (issuer) {
+        tma_store_2d(map, 0, y, stage_base);
+        if (nh > 1) tma_store_2d(map, 0, y + 64, stage_base + 64 * 128);
+        bulk_commit();
+        bulk_wait_read_all();
+      }
+      named_sync(2, 128);
+    };
     while (it.next(j)) {
       const int a = n & 1;
-      if (!warp_ok(mbar_wait(&bar->g_full[a], (uint32_t)(n >> 1) & 1u, abort, status))) break;
+      const bool got = mbar_wait(&bar->g_full[a], (uint32_t)(n >> 1) & 1u, abort, status);
+      if (!group_ok(2, 128, got)) break;
       tc_fence_after();
       const int nc = min(3, n_chunks - 2 * j.p);
-      const int64_t bh = j.seg / n_rounds;
-      const int* tk = bar->tok[n & 3];
-      const int tok = row < 64 * min(nc, 2) ? tk[row] : -1;
+      const int nh = min(nc, 2);                 // 64-row halves of key rows present
+      const int y = (int)(j.seg * L) + 2 * j.p * kM;
       const uint32_t acc = tl + kColAcc + (uint32_t)a * 128;
-      flush_rows(dv + bh * L * 64, tok, acc, 1.f, stage, lane);
-      flush_rows(dqk + bh * L * 64, tok, acc + 64, scale, stage, lane);
-      if (j.last && nc == 3 && q < 2) {
-        // R1 rows (chunk 2p+2) that no later item of this unit picks up
-        flush_rows(dqk + bh * L * 64, tk[128 + row], tl + kColAcc + (uint32_t)(a ^ 1) * 128 + 64,
-                   scale, stage, lane);
+      const bool r1 = j.last && nc == 3;
+      stage_row(acc, 1.f, stage_base, row);
+      store_rows(&map_dv, y, nh);
+      stage_row(acc + 64, scale, stage_base, row);
+      if (!r1) {
+        tc_fence_before();
+        mbar_arrive(&bar->acc_free[a]);
       }
-      tc_fence_before();
-      mbar_arrive(&bar->acc_free[a]);
+      store_rows(&map_dqk, y, nh);
+      if (r1) {
+        // R1 rows (chunk 2p+2) that no later item of this unit picks up
+        if (q < 2) stage_row(tl + kColAcc + (uint32_t)(a ^ 1) * 128 + 64, scale, stage_base, row);
+        tc_fence_before();
+        mbar_arrive(&bar->acc_free[a]);
+        store_rows(&map_edge, (int)(j.seg * units_per_seg + j.p / kUnit) * kM, 1);
+      }
       ++n;
     }
+    if (issuer) bulk_wait_all();
   } else {
     // ------------------------------------------------ softmax: P^T and dS^T
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSmx));
@@ -548,8 +577,10 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
                 dk[2 * i4] = pack_f16x2(de[0], de[1]);
                 dk[2 * i4 + 1] = pack_f16x2(de[2], de[3]);
               }
-              // P^T over the S^T columns already read; dS^T into shared memory
+              // P^T and dS^T over the S^T / dP^T columns already read; dS^T
+              // also into shared memory
               tmem_st16(tb + h * 16, pk);
+              tmem_st16(tb + 64 + h * 16, dk);
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
                 const int ch = h * 4 + c;
@@ -563,6 +594,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
 #pragma unroll
             for (int e = 0; e < 32; ++e) z[e] = 0u;
             tmem_st32(tb, z);
+            tmem_st32(tb + 64, z);
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch)
               *reinterpret_cast<uint4*>(drow + ((ch ^ (row & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
@@ -584,17 +616,148 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
   }
 }
 
+// inv[seg][perm[seg][i]] = i: the slot of every position in every round.
+__global__ void __launch_bounds__(256)
+inverse_perm_kernel(const int32_t* __restrict__ perm, int32_t* __restrict__ inv, int L,
+                    int64_t total, int* status) {
+  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= total) return;
+  const int64_t seg = k / L;
+  const int i = (int)(k - seg * L);
+  const int pos = perm[k];
+  if ((unsigned)pos >= (unsigned)L) {
+    if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
+    return;
+  }
+  inv[seg * L + pos] = i;
+}
+
+__device__ __forceinline__ void add8_f16(float (&acc)[8], const __half* src) {
+  const uint4 w = *reinterpret_cast<const uint4*>(src);
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
+    acc[2 * i] += f.x;
+    acc[2 * i + 1] += f.y;
+  }
+}
+
+// dv, dqk of every token: the sum over rounds of its partial rows (slot
+// inv[seg][pos] of segment seg = bh * n_rounds + r), plus the unit-end R1
+// row where its slot opens a unit; dv also takes dout for a token that
+// attended only to itself (final LSE of -inf). Eight threads per token.
+__global__ void __launch_bounds__(256)
+unsort_kernel(const __half* __restrict__ part_dv, const __half* __restrict__ part_dqk,
+              const __half* __restrict__ edge, const int32_t* __restrict__ inv,
+              const float* __restrict__ lse, const __nv_bfloat16* __restrict__ dout,
+              float* __restrict__ dqk, float* __restrict__ dv, int L, int n_rounds,
+              int units_per_seg, int64_t N, int* status) {
+  const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
+  const int c8 = (threadIdx.x & 7) * 8;
+  if (t >= N) return;
+  const int64_t bh = t / L;
+  const int pos = (int)(t - bh * L);
+  float a[8], b[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) a[e] = b[e] = 0.f;
+  for (int r = 0; r < n_rounds; ++r) {
+    const int64_t seg = bh * n_rounds + r;
+    const int i = inv[seg * L + pos];
+    if ((unsigned)i >= (unsigned)L) {
+      if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
+      continue;
+    }
+    const int64_t row = seg * L + i;
+    add8_f16(a, part_dv + row * 64 + c8);
+    add8_f16(b, part_dqk + row * 64 + c8);
+    const int c = i / kM;
+    if (c > 0 && c % (2 * kUnit) == 0) {
+      const int64_t er = (seg * units_per_seg + c / (2 * kUnit) - 1) * kM + (i % kM);
+      add8_f16(b, edge + er * 64 + c8);
+    }
+  }
+  if (lse[t] == -INFINITY) {
+    const uint4 w = *reinterpret_cast<const uint4*>(dout + t * 64 + c8);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      a[2 * i] += __uint_as_float(u[i] << 16);
+      a[2 * i + 1] += __uint_as_float(u[i] & 0xffff0000u);
+    }
+  }
+  float4* pv = reinterpret_cast<float4*>(dv + t * 64 + c8);
+  float4* pq = reinterpret_cast<float4*>(dqk + t * 64 + c8);
+  pv[0] = make_float4(a[0], a[1], a[2], a[3]);
+  pv[1] = make_float4(a[4], a[5], a[6], a[7]);
+  pq[0] = make_float4(b[0], b[1], b[2], b[3]);
+  pq[1] = make_float4(b[4], b[5], b[6], b[7]);
+}
+
+bool tc_eligible(const lsh_problem& p) {
+  if (p.dtype != LSH_BF16 || p.chunk != kM || !(p.scale > 0.f) || p.L % kM != 0) return false;
+  const int n_pairs = (p.L / kM + 1) / 2;
+  const int64_t units = (int64_t)p.B * p.H * p.n_rounds * ((n_pairs + kUnit - 1) / kUnit);
+  const int64_t rows = (int64_t)p.B * p.H * p.n_rounds * p.L;
+  return units <= INT32_MAX && rows <= INT32_MAX;
+}
+
+struct TcWs {
+  int32_t* inv;
+  __half* part_dv;
+  __half* part_dqk;
+  __half* edge;
+  size_t bytes;
+};
+TcWs tc_ws(const lsh_problem& p, void* base) {
+  const size_t rows = (size_t)p.B * p.H * p.n_rounds * p.L;
+  const int n_pairs = (p.L / kM + 1) / 2;
+  const size_t edge_rows =
+      (size_t)p.B * p.H * p.n_rounds * ((n_pairs + kUnit - 1) / kUnit) * kM;
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  TcWs w;
+  char* c = (char*)base;
+  size_t off = 0;
+  w.inv = (int32_t*)(c + off);
+  off += al(rows * 4);
+  w.part_dv = (__half*)(c + off);
+  off += al(rows * 64 * 2);
+  w.part_dqk = (__half*)(c + off);
+  off += al(rows * 64 * 2);
+  w.edge = (__half*)(c + off);
+  off += al(edge_rows * 64 * 2);
+  w.bytes = off;
+  return w;
+}
+
 }  // namespace
+
+size_t bwd_tc_ws_bytes(const lsh_problem& p) {
+  return tc_eligible(p) ? tc_ws(p, nullptr).bytes : 0;
+}
 
 cudaError_t launch_attn_bwd_tc(const lsh_problem& p, const void* qk, const void* v,
                                const void* dout, const int32_t* perm, const float* lse,
-                               const float* D, float* dqk, float* dv, int* status, cudaStream_t s) {
-  if (p.dtype != LSH_BF16 || p.chunk != kM || !(p.scale > 0.f)) return cudaErrorNotSupported;
+                               const float* D, float* dqk, float* dv, void* ws, int* status,
+                               cudaStream_t s) {
+  if (!tc_eligible(p)) return cudaErrorNotSupported;
+  const TcWs w = tc_ws(p, ws);
   const int n_chunks = p.L / kM;
   const int n_pairs = (n_chunks + 1) / 2;
   const int units_per_seg = (n_pairs + kUnit - 1) / kUnit;
-  const int64_t n_units = (int64_t)p.B * p.H * p.n_rounds * units_per_seg;
-  if (n_units > INT32_MAX) return cudaErrorNotSupported;
+  const int64_t n_segs = (int64_t)p.B * p.H * p.n_rounds;
+  const int64_t n_units = n_segs * units_per_seg;
+  const int64_t rows = n_segs * p.L;
+  const int64_t N = (int64_t)p.B * p.H * p.L;
+  // per-round partial gradients (fp16 rows in slot order) and unit-end R1 rows,
+  // written by 64-row TMA boxes with 128-byte swizzle
+  CUtensorMap m_dv, m_dqk, m_edge;
+  if (!encode_tmap_2d_16bit(&m_dv, w.part_dv, 64, (uint64_t)rows, 128, 64, 64) ||
+      !encode_tmap_2d_16bit(&m_dqk, w.part_dqk, 64, (uint64_t)rows, 128, 64, 64) ||
+      !encode_tmap_2d_16bit(&m_edge, w.edge, 64, (uint64_t)(n_units * kM), 128, 64, 64))
+    return cudaErrorInvalidValue;
+  inverse_perm_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(perm, w.inv, p.L, rows,
+                                                                      status);
   int grid = sm_count();
   if ((int64_t)grid > n_units) grid = (int)n_units;
   auto kern = p.causal ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
@@ -603,8 +766,12 @@ cudaError_t launch_attn_bwd_tc(const lsh_problem& p, const void* qk, const void*
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemBytes, s>>>(
       (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, (const __nv_bfloat16*)dout, perm, lse, D,
-      dqk, dv, p.L, p.n_rounds, p.scale, p.scale * kLog2e, (int)n_units, units_per_seg, status);
-  note_launch();
+      m_dv, m_dqk, m_edge, p.L, p.n_rounds, p.scale, p.scale * kLog2e, (int)n_units,
+      units_per_seg, status);
+  unsort_kernel<<<(unsigned)((N * 8 + 255) / 256), 256, 0, s>>>(
+      w.part_dv, w.part_dqk, w.edge, w.inv, lse, (const __nv_bfloat16*)dout, dqk, dv, p.L,
+      p.n_rounds, units_per_seg, N, status);
+  note_launch(3);
   return cudaGetLastError();
 }
 

@@ -288,12 +288,13 @@ combine_f16_kernel(const __half* __restrict__ opart, const float* __restrict__ l
   if (c8 == 0) lse[tok] = LSE;
 }
 
-// D_i = dout_i . out_i; zero dqk; dv = dout for self-attending rows, else 0.
+// D_i = dout_i . out_i; with init_grads also zero dqk and set dv = dout for
+// self-attending rows, else 0.
 template <typename T>
 __global__ void __launch_bounds__(256)
 bwd_prep_kernel(const T* __restrict__ out, const T* __restrict__ out_lo, const T* __restrict__ dout,
                 const float* __restrict__ lse, float* __restrict__ D, float* __restrict__ dqk,
-                float* __restrict__ dv, int64_t N) {
+                float* __restrict__ dv, int64_t N, bool init_grads) {
   const int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
   const int c4 = (threadIdx.x & 15) * 4;
   const bool live = tok < N;
@@ -309,6 +310,7 @@ bwd_prep_kernel(const T* __restrict__ out, const T* __restrict__ out_lo, const T
   float d = warp_sum16(o.x * g.x + o.y * g.y + o.z * g.z + o.w * g.w);
   if (!live) return;
   if (c4 == 0) D[tok] = d;
+  if (!init_grads) return;
   const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
   store4(dqk + tok * kD + c4, z);
   store4(dv + tok * kD + c4, lse[tok] == -INFINITY ? g : z);
@@ -498,11 +500,15 @@ cudaError_t bwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* 
   cudaError_t e = cudaFuncSetAttribute(bwd_round_kernel<T>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem);
   if (e != cudaSuccess) return e;
+  const bool tc = bwd_tc_ws_bytes(p) > 0;
   bwd_prep_kernel<T><<<(unsigned)((N * 16 + 255) / 256), 256, 0, s>>>(out, out_lo, dout, lse, D, dqk, dv,
-                                                                        N);
+                                                                        N, !tc);
   note_launch();
-  e = launch_attn_bwd_tc(p, qk, v, dout, perm, lse, D, dqk, dv, status, s);
-  if (e != cudaErrorNotSupported) return e == cudaSuccess ? cudaGetLastError() : e;
+  if (tc) {
+    e = launch_attn_bwd_tc(p, qk, v, dout, perm, lse, D, dqk, dv,
+                           (char*)D + align_up((size_t)N * 4, 256), status, s);
+    return e == cudaSuccess ? cudaGetLastError() : e;
+  }
   bwd_round_kernel<T><<<(unsigned)blocks, 256, kBwdSmem, s>>>(
       qk, v, dout, perm, lse, D, dqk, dv, p.L, p.chunk, p.n_rounds, p.causal, p.scale,
       p.scale * kLog2e, status);
@@ -536,7 +542,7 @@ cudaError_t launch_attn_fwd(const lsh_problem& p, const void* qk, const void* v,
 }
 
 size_t bwd_ws_bytes(const lsh_problem& p) {
-  return align_up((size_t)p.B * p.H * p.L * 4, 256);
+  return align_up((size_t)p.B * p.H * p.L * 4, 256) + bwd_tc_ws_bytes(p);
 }
 
 cudaError_t launch_attn_bwd(const lsh_problem& p, const void* qk, const void* v,

@@ -54,11 +54,16 @@ cudaError_t launch_attn_fwd_tc(const lsh_problem& p, const void* qk, const void*
                                const int32_t* perm, void* opart_f16, float* lsepart, int* status,
                                cudaStream_t s);
 
-// tcgen05 backward (bf16, chunk 64): accumulates into dqk/dv, which must hold
-// the initial values (zeros, dout for self-attending rows); D = dout . out.
+// tcgen05 backward (bf16, chunk 64): writes dqk and dv (every element, the
+// self-attending rows' dout included) from D = dout . out; `ws` holds
+// bwd_tc_ws_bytes(p) bytes (inverse permutation, per-round fp16 partials).
+// bwd_tc_ws_bytes is 0 and the launcher returns cudaErrorNotSupported for
+// other problems.
+size_t bwd_tc_ws_bytes(const lsh_problem& p);
 cudaError_t launch_attn_bwd_tc(const lsh_problem& p, const void* qk, const void* v,
                                const void* dout, const int32_t* perm, const float* lse,
-                               const float* D, float* dqk, float* dv, int* status, cudaStream_t s);
+                               const float* D, float* dqk, float* dv, void* ws, int* status,
+                               cudaStream_t s);
 
 size_t bwd_ws_bytes(const lsh_problem& p);
 cudaError_t launch_attn_bwd(const lsh_problem& p, const void* qk, const void* v,

@@ -105,6 +105,29 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ---------------------------------------------------------------- TMA store
+// Tiled shared -> global copy of one box at element coordinates (x, y) of a
+// 2D tensor map (x a multiple of 16 bytes' worth of elements; y >= 0); boxes
+// reaching past the tensor's extent are clipped. Tracked per thread in bulk
+// groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int32_t x, int32_t y,
+                                             const void* src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+               ::"l"((uint64_t)map), "r"(x), "r"(y), "r"(smem_u32(src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until the shared-memory sources of all committed bulk groups have been read.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Waits until all committed bulk groups have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // In-place bf16 -> fp16 conversion of one 16-byte piece of shared memory
 // (8 elements; exact for bf16 values inside the fp16 range).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
