@@ -12,19 +12,19 @@
 // Structure (one CTA per SM, persistent; CTAs are assigned to one round so
 // that R_r stays resident in shared memory):
 //   warp 0  : TMA producer — R_r once (MN-major operand), then 128-token X
-//             tiles (K-major) through a 4-stage ring;
-//   warp 1  : TMEM allocation; one thread issues tcgen05.mma: a 128 x N x 64
-//             product per 256-column chunk of R_r into one of two TMEM
-//             accumulators (so the epilogue of one chunk overlaps the MMA of
-//             the next);
-//   warps 2-5: epilogue — tcgen05.ld of the accumulator rows (one token per
-//             thread). Each |s| becomes a float key whose 4 low mantissa bits
-//             hold (15 - its 32-column group), so one 3-input max folds two
-//             columns into each of 32 per-position running maxima with the
-//             lowest column winning ties; values closer than 2^-19 relative
-//             count as ties (a near-tie by the 1e-5 bound the results are
-//             checked against). The winner's sign is recomputed from the X and
-//             R tiles in shared memory, then the bucket id is written.
+//             tiles (K-major) through a 4-stage ring, released by the MMAs;
+//   warp 1  : TMEM allocation; one thread issues tcgen05.mma: a 128 x 256 x 64
+//             product per 256-column chunk of R_r;
+//   warps 2-5, 6-9: two epilogue warpgroups taking alternate tiles, each with
+//             its own 256-column TMEM accumulator (one token per thread).
+//             Each s becomes a float key whose 4 low mantissa bits hold
+//             (15 - its 32-column group) and whose sign is kept; two 3-input
+//             max and min operations fold two columns into each of 32
+//             per-position running maxima (largest +s) and minima (most
+//             negative s), the lowest column winning ties. Values closer than
+//             2^-19 relative count as ties (a near-tie by the 1e-5 bound the
+//             results are checked against). The merge picks the larger of the
+//             best +s and the best -s, the +s half first on ties.
 // Handles n_b/2 <= 512 with n_b/2 a multiple of 8; other shapes use the
 // CUDA-core kernel.
 #include "common.cuh"
@@ -44,7 +44,7 @@ constexpr int kChunkN = 256;         // columns per MMA / accumulator
 constexpr int kXBytes = kTileM * 128;              // 16 KB
 constexpr int kRBlockBytes = 64 * 128;             // 64 columns x 64 k-rows
 constexpr int kRBytes = (kMaxNh / 64) * kRBlockBytes;  // 64 KB
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 
 struct __align__(8) HashBarriers {
   uint64_t r_full;
@@ -58,6 +58,21 @@ struct __align__(8) HashBarriers {
 };
 
 constexpr size_t kSmemBytes = 1024 + kRBytes + kStages * kXBytes + sizeof(HashBarriers);
+
+__device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
+
+// Folds two accumulator values (raw fp32 bits a, b; group tags ta, tb in the
+// low 4 mantissa bits) into the running maximum and minimum of one position.
+__device__ __forceinline__ void fold2(float& mx, float& mn, uint32_t a, uint32_t b, uint32_t ta,
+                                      uint32_t tb) {
+  const float ka = __uint_as_float((a & 0xFFFFFFF0u) | ta);
+  const float kb = __uint_as_float((b & 0xFFFFFFF0u) | tb);
+  float r0, r1;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r0) : "f"(mx), "f"(ka), "f"(kb));
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r1) : "f"(mn), "f"(ka), "f"(kb));
+  mx = r0;
+  mn = r1;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_r,
@@ -80,7 +95,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     mbar_init(&bar->r_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar->x_full[s], 1);
-      mbar_init(&bar->x_empty[s], 128);   // released by the epilogue (sign recompute)
+      mbar_init(&bar->x_empty[s], 1);     // released by the MMAs' commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar->acc_full[b], 1);
@@ -128,38 +143,47 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
+      // Tiles alternate between the two accumulators / epilogue warpgroups;
+      // the chunks of a pair of tiles are interleaved so both stay busy.
       if (mbar_wait(&bar->r_full, 0, abort, status)) {
         tc_fence_after();
         const uint32_t r_base = smem_u32(r_smem);
         const uint32_t x_base = smem_u32(x_smem);
-        int it = 0, job = 0;
+        int uses[2] = {0, 0};
         bool ok = true;
-        for (int t = ci; t < n_tiles && ok; t += ctas_per_round, ++it) {
-          const int s = it % kStages;
-          if (!mbar_wait(&bar->x_full[s], (uint32_t)(it / kStages) & 1u, abort, status)) break;
+        auto issue = [&](int it, int j) -> bool {
+          const int w = it & 1, s = it % kStages;
+          if (uses[w] > 0 &&
+              !mbar_wait(&bar->acc_empty[w], (uint32_t)(uses[w] - 1) & 1u, abort, status))
+            return false;
+          ++uses[w];
           tc_fence_after();
-          for (int j = 0; j < nsub; ++j, ++job) {
-            const int buf = job & 1;
-            const int use = job >> 1;
-            if (use > 0 && !mbar_wait(&bar->acc_empty[buf], (uint32_t)(use - 1) & 1u, abort, status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const int ncols = min(kChunkN, nh - j * kChunkN);
-            // whole 64-column blocks: the MN-major operand is read in complete
-            // swizzle atoms; the zero-filled extra columns are masked later
-            const int n_mma = (ncols + 63) / 64 * 64;
-            const uint32_t idesc = idesc_f16(kTileM, n_mma, 1, false, true);
-            const uint32_t d = tmem + (uint32_t)(buf * kChunkN);
+          const int ncols = min(kChunkN, nh - j * kChunkN);
+          // whole 64-column blocks: the MN-major operand is read in complete
+          // swizzle atoms; the zero-filled extra columns are masked later
+          const int n_mma = (ncols + 63) / 64 * 64;
+          const uint32_t idesc = idesc_f16(kTileM, n_mma, 1, false, true);
+          const uint32_t d = tmem + (uint32_t)(w * kChunkN);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              uint64_t a = smem_desc(x_base + s * kXBytes + k * 32, 16, 1024);
-              uint64_t b = smem_desc(r_base + j * 4 * kRBlockBytes + k * 2048, kRBlockBytes, 1024);
-              mma_ss(d, a, b, idesc, k > 0 ? 1u : 0u);
-            }
-            mma_commit(&bar->acc_full[buf]);
+          for (int k = 0; k < 4; ++k) {
+            uint64_t a = smem_desc(x_base + s * kXBytes + k * 32, 16, 1024);
+            uint64_t b = smem_desc(r_base + j * 4 * kRBlockBytes + k * 2048, kRBlockBytes, 1024);
+            mma_ss(d, a, b, idesc, k > 0 ? 1u : 0u);
           }
+          mma_commit(&bar->acc_full[w]);
+          if (j == nsub - 1) mma_commit(&bar->x_empty[s]);
+          return true;
+        };
+        const int n_mine = (n_tiles - ci + ctas_per_round - 1) / ctas_per_round;
+        for (int it0 = 0; it0 < n_mine && ok; it0 += 2) {
+          const int cnt = min(2, n_mine - it0);
+          for (int k = 0; k < cnt && ok; ++k)
+            ok = mbar_wait(&bar->x_full[(it0 + k) % kStages],
+                           (uint32_t)((it0 + k) / kStages) & 1u, abort, status);
+          if (!ok) break;
+          tc_fence_after();
+          for (int j = 0; j < nsub && ok; ++j)
+            for (int k = 0; k < cnt && ok; ++k) ok = issue(it0 + k, j);
         }
       }
       // all issued MMAs have finished before TMEM is released (bounded)
@@ -168,80 +192,74 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
       mbar_wait(&bar->mma_done, 0, (volatile int*)&dummy, status);
     }
   } else {
-    // ---------------- epilogue: warps 2..5 ----------------
+    // ---------------- epilogue: warps 2..5 and 6..9 ----------------
+    const int w = (warp - 2) >> 2;          // warpgroup = accumulator = tile parity
     const int q = warp & 3;                 // TMEM lane quarter this warp may read
     const int row_in_tile = q * 32 + lane;
-    int job = 0, it = 0;
+    const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(w * kChunkN);
+    int use = 0, it = 0;
     bool ok = true;
     for (int t = ci; t < n_tiles && ok; t += ctas_per_round, ++it) {
-      float acc[32];
+      if ((it & 1) != w) continue;
+      float mx[32], mn[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+      for (int i = 0; i < 32; ++i) {
+        mx[i] = -INFINITY;
+        mn[i] = INFINITY;
+      }
       int g = 0;                              // global 32-column group index
-      for (int j = 0; j < nsub; ++j, ++job) {
-        const int buf = job & 1;
-        if (!mbar_wait(&bar->acc_full[buf], (uint32_t)(job >> 1) & 1u, abort, status)) {
+      for (int j = 0; j < nsub; ++j, ++use) {
+        if (!warp_all(mbar_wait(&bar->acc_full[w], (uint32_t)use & 1u, abort, status))) {
           ok = false;
           break;
         }
         tc_fence_after();
         const int ncols = min(kChunkN, nh - j * kChunkN);
-        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kChunkN);
         for (int c0 = 0; c0 < ncols; c0 += 64, g += 2) {
           uint32_t va[32], vb[32];
-          tmem_ld32(taddr + c0, va);
-          tmem_ld32(taddr + c0 + 32, vb);     // within the 512 allocated columns
+          tmem_ld32(tbase + c0, va);
+          tmem_ld32(tbase + c0 + 32, vb);     // within the accumulator's 256 columns
           tmem_ld_wait();
           const uint32_t ma = (uint32_t)(15 - g), mb = (uint32_t)(14 - g);
-          const int na = min(32, ncols - c0), nb = min(32, ncols - c0 - 32);
+          if (ncols - c0 >= 64) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const uint32_t ka = (i < na) ? ((va[i] & 0x7FFFFFF0u) | ma) : 0u;
-            const uint32_t kb = (i < nb) ? ((vb[i] & 0x7FFFFFF0u) | mb) : 0u;
-            float r;
-            asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(acc[i]), "f"(__uint_as_float(ka)),
-                "f"(__uint_as_float(kb)));
-            acc[i] = r;
+            for (int i = 0; i < 32; ++i) fold2(mx[i], mn[i], va[i], vb[i], ma, mb);
+          } else {
+            const int na = ncols - c0, nb = ncols - c0 - 32;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              // a missing column is a NaN key, which max and min ignore
+              const uint32_t a = (i < na) ? va[i] : 0x7FFFFFFFu;
+              const uint32_t b = (i < nb) ? vb[i] : 0x7FFFFFFFu;
+              fold2(mx[i], mn[i], a, b, ma, mb);
+            }
           }
         }
         tc_fence_before();
-        mbar_arrive(&bar->acc_empty[buf]);
+        mbar_arrive(&bar->acc_empty[w]);
       }
       if (!ok) break;
-      // merge: largest key magnitude, smallest column on ties
+      // merge: largest |s| over both halves; on ties the +s half, then the
+      // smaller column
       uint32_t best_m = 0;
       int best_c = 0x7fffffff;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const uint32_t k = __float_as_uint(acc[i]);
-        const uint32_t m = k & 0x7FFFFFF0u;
-        const int c = (15 - (int)(k & 15u)) * 32 + i;
-        if (m > best_m || (m == best_m && c < best_c)) { best_m = m; best_c = c; }
+        const uint32_t kp = __float_as_uint(mx[i]), kn = __float_as_uint(mn[i]);
+        // a negative running maximum or a positive running minimum (this
+        // includes the initial -inf / +inf) is never the winner
+        const bool vp = (kp >> 31) == 0u, vq = (kn >> 31) != 0u;
+        const uint32_t mp = vp ? (kp & 0x7FFFFFF0u) : 0u;
+        const int cp = vp ? (15 - (int)(kp & 15u)) * 32 + i : 0x7fffffff;
+        const uint32_t mq = vq ? (kn & 0x7FFFFFF0u) : 0u;
+        const int cq = vq ? nh + (15 - (int)(kn & 15u)) * 32 + i : 0x7fffffff;
+        if (mp > best_m || (mp == best_m && cp < best_c)) { best_m = mp; best_c = cp; }
+        if (mq > best_m || (mq == best_m && cq < best_c)) { best_m = mq; best_c = cq; }
       }
-      // sign of s at the winning column: x . R[:, col] from shared memory
-      const int s_idx = it % kStages;
-      const uint8_t* xrow = x_smem + s_idx * kXBytes + row_in_tile * 128;
-      const uint8_t* rblk = r_smem + (best_c >> 6) * kRBlockBytes;
-      const int nn = best_c & 63;
-      float dot = 0.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 w = *reinterpret_cast<const uint4*>(xrow + (((uint32_t)c ^ (uint32_t)(row_in_tile & 7)) << 4));
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int k = c * 8 + e;
-          const float xv = __uint_as_float((e & 1) ? (ws[e >> 1] & 0xffff0000u) : (ws[e >> 1] << 16));
-          const uint16_t rb = *reinterpret_cast<const uint16_t*>(
-              rblk + k * 128 + ((((uint32_t)nn >> 3) ^ (uint32_t)(k & 7)) << 4) + (nn & 7) * 2);
-          dot = fmaf(xv, __uint_as_float((uint32_t)rb << 16), dot);
-        }
-      }
-      mbar_arrive(&bar->x_empty[s_idx]);
       const int64_t row = (int64_t)t * kTileM + row_in_tile;
       if (row < n_rows) {
         const int64_t bh = row / L, pos = row - bh * L;
-        bucket[(bh * n_rounds + r) * L + pos] = dot >= 0.f ? best_c : nh + best_c;
+        bucket[(bh * n_rounds + r) * L + pos] = best_c;
       }
     }
   }
