@@ -201,6 +201,52 @@ __device__ __forceinline__ void stage_row(uint32_t ta, float sc, uint8_t* stage,
   }
 }
 
+// ---- MMA issue helpers (one thread). Descriptor lower words: `sl` is the
+// slot's shared address >> 4; LBO fields are added per operand layout.
+constexpr uint32_t kIdKK = idesc_f16(128, 64, 0, false, false);   // A, B K-major
+constexpr uint32_t kIdKN = idesc_f16(128, 64, 0, false, true);    // B MN-major
+constexpr uint32_t kIdNN = idesc_f16(128, 64, 0, true, true);     // A, B MN-major
+constexpr uint32_t kLboK = desc_lbo(16), kLboN = desc_lbo(kTile);
+
+// S^T = X_K X_qb^T and dP^T = V_K dO_qb^T of step g (buffer g & 1); commits `full`.
+__device__ __forceinline__ void bwd_issue_s(uint32_t tmem, uint32_t sl, int g, int qb, int nc,
+                                            uint64_t* full) {
+  if (qb < nc) {
+    const uint32_t d = tmem + kColBuf + (uint32_t)(g & 1) * 128;
+    const uint32_t xk = sl + kX / 16 + kLboK, vk = sl + kV / 16 + kLboK;
+    const uint32_t xq = sl + (kX + qb * kTile) / 16 + kLboK, gq = sl + (kDo + qb * kTile) / 16 + kLboK;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      mma_ss_w(d, xk + 2 * ks, xq + 2 * ks, kDescHi1024, kIdKK, ks > 0);
+      mma_ss_w(d + 64, vk + 2 * ks, gq + 2 * ks, kDescHi1024, kIdKK, ks > 0);
+    }
+  }
+  mma_commit(full);
+}
+// dV += P^T dO_qb ; dK += dS^T X_qb, P^T and dS^T from step g's TMEM buffer.
+__device__ __forceinline__ void bwd_issue_g(uint32_t tmem, uint32_t acc, uint32_t sl, int g, int qb,
+                                            bool acc_v, bool acc_k) {
+  const uint32_t pt = tmem + kColBuf + (uint32_t)(g & 1) * 128;
+  const uint32_t gq = sl + (kDo + qb * kTile) / 16 + kLboN, xq = sl + (kX + qb * kTile) / 16 + kLboN;
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    mma_ts_w(acc, pt + ks * 8, gq + 128 * ks, kDescHi1024, kIdKN, acc_v || ks > 0);
+    mma_ts_w(acc + 64, pt + 64 + ks * 8, xq + 128 * ks, kDescHi1024, kIdKN, acc_k || ks > 0);
+  }
+}
+// Query-side product dS[128 queries of the dS^T blocks at ds] X_K over the
+// first 16 KS keys, into the dK columns at d.
+template <int KS>
+__device__ __forceinline__ void bwd_issue_r(uint32_t d, uint32_t ds, uint32_t sl, bool acc) {
+  const uint32_t xk = sl + kX / 16 + kLboN;
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks)
+    mma_ss_w(d, ds + 128 * ks, xk + 128 * ks, kDescHi1024, kIdNN, acc || ks > 0);
+}
+__device__ __forceinline__ bool bwd_wait_p(BwdBar* bar, int g, volatile int* abort, int* status) {
+  return mbar_wait(&bar->p_full[g & 1], (uint32_t)(g >> 1) & 1u, abort, status);
+}
+
 template <bool kCausal>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __restrict__ v,
@@ -347,66 +393,20 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
       }
     } else if (lane == 0) {
       // ---------------------------------------------- MMA issuer
-      const uint32_t idesc_kk = idesc_f16(128, 64, 0, false, false);   // both K-major
-      const uint32_t idesc_kn = idesc_f16(128, 64, 0, false, true);    // B MN-major
-      const uint32_t idesc_nn = idesc_f16(128, 64, 0, true, true);     // A and B MN-major
-      const uint32_t slots_a = smem_u32(slots), ds_a = smem_u32(dsb);
-      // descriptor templates (start address 0); a shared-memory address below
-      // 256 KB is added to the 14-bit start-address field as addr >> 4
-      const uint64_t t_k = smem_desc(0, 16, 1024);        // K-major
-      const uint64_t t_n = smem_desc(0, kTile, 1024);     // MN-major input tile
-      const uint64_t t_d = smem_desc(0, kDsBlock, 1024);  // MN-major reading of dS^T
-      auto dsc = [](uint64_t t, uint32_t addr) { return t + (uint64_t)(addr >> 4); };
-      int acc_seen[2] = {0, 0};
-      // waits until the flushes of the first `need` items that used set `a` are done
-      auto wait_acc = [&](int a, int need) -> bool {
-        while (acc_seen[a] < need) {
-          if (!mbar_wait(&bar->acc_free[a], (uint32_t)acc_seen[a] & 1u, abort, status))
-            return false;
-          ++acc_seen[a];
-        }
-        return true;
-      };
-      // S^T and dP^T of step (item nn, query block qb) into buffer (3 nn + qb) & 1
-      auto issue_s = [&](int nn, int qb, int nc, uint32_t sl) {
-        const int w = (3 * nn + qb) & 1;
-        if (qb < nc) {
-          const uint32_t d = tmem + kColBuf + (uint32_t)w * 128;
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            mma_ss(d, dsc(t_k, sl + kX + ks * 32),
-                   dsc(t_k, sl + kX + qb * kTile + ks * 32), idesc_kk, ks > 0);
-            mma_ss(d + 64, dsc(t_k, sl + kV + ks * 32),
-                   dsc(t_k, sl + kDo + qb * kTile + ks * 32), idesc_kk, ks > 0);
-          }
-        }
-        mma_commit(&bar->s_full[w]);
-      };
-      auto wait_p = [&](int g) {
-        return mbar_wait(&bar->p_full[g & 1], (uint32_t)(g >> 1) & 1u, abort, status);
-      };
-      // dV += P^T dO_qb ; dK += dS^T_qb X_qb (P^T and dS^T from TMEM)
-      auto issue_g = [&](int g, int qb, uint32_t sl, uint32_t acc, bool acc_v, bool acc_k) {
-        const uint32_t pt = tmem + kColBuf + (uint32_t)(g & 1) * 128;
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          mma_ts(acc, pt + ks * 8, dsc(t_n, sl + kDo + qb * kTile + ks * 2048),
-                 idesc_kn, acc_v || ks > 0);
-          mma_ts(acc + 64, pt + 64 + ks * 8, dsc(t_n, sl + kX + qb * kTile + ks * 2048),
-                 idesc_kn, acc_k || ks > 0);
-        }
-      };
       JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
       Job cur, nxt;
       bool have = it.next(cur);
       bool ok = true;
+      const uint32_t slot0 = smem_u32(slots) >> 4;
+      const uint32_t ds_lo = (smem_u32(dsb) >> 4) | desc_lbo(kDsBlock);
+      int seen0 = 0, seen1 = 0;   // acc_free completions waited for, per set
       if (have) {
         ok = mbar_wait(&bar->slot_full[0], 0u, abort, status);
         if (ok) {
           tc_fence_after();
           const int nc = min(3, n_chunks - 2 * cur.p);
-          issue_s(0, 0, nc, slots_a);
-          issue_s(0, 1, nc, slots_a);
+          bwd_issue_s(tmem, slot0, 0, 0, nc, &bar->s_full[0]);
+          bwd_issue_s(tmem, slot0, 1, 1, nc, &bar->s_full[1]);
         }
       }
       int n = 0;
@@ -415,23 +415,34 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
         const bool have_next = it.next(nxt);
         const int s = n % kSlots, a = n & 1;
         const int nc = min(3, n_chunks - 2 * cur.p);
-        const uint32_t sl = slots_a + s * kSlotBytes;
+        const uint32_t sl = slot0 + (uint32_t)(s * kSlotBytes) / 16;
         const uint32_t acc = tmem + kColAcc + (uint32_t)a * 128;
         const int g0 = 3 * n;
         // ---- block 0 (always present)
-        if (!wait_p(g0) || !wait_acc(a, n >> 1)) break;
-        if (prev_r1_alone && !wait_acc(a ^ 1, ((n - 1) >> 1) + 1)) break;
+        if (!bwd_wait_p(bar, g0, abort, status)) break;
+        // flushes of the earlier items that used set a (and, after a unit's
+        // last item, of that item too: it read its R1 rows from set a)
+        {
+          const int need = n >> 1;
+          int& seen = a ? seen1 : seen0;
+          while (ok && seen < need) ok = mbar_wait(&bar->acc_free[a], (uint32_t)(seen++) & 1u, abort, status);
+          if (prev_r1_alone) {
+            const int b = a ^ 1, need_b = ((n - 1) >> 1) + 1;
+            int& seen_b = b ? seen1 : seen0;
+            while (ok && seen_b < need_b)
+              ok = mbar_wait(&bar->acc_free[b], (uint32_t)(seen_b++) & 1u, abort, status);
+          }
+          if (!ok) break;
+        }
         tc_fence_after();
-        issue_g(g0, 0, sl, acc, false, !cur.first);
-        issue_s(n, 2, nc, sl);
+        bwd_issue_g(tmem, acc, sl, g0, 0, false, !cur.first);
+        bwd_issue_s(tmem, sl, g0 + 2, 2, nc, &bar->s_full[(g0 + 2) & 1]);
         // ---- block 1, then R0 = dS[blocks 0,1] X_K into dK
-        if (!wait_p(g0 + 1)) break;
+        if (!bwd_wait_p(bar, g0 + 1, abort, status)) break;
         tc_fence_after();
-        if (nc > 1) issue_g(g0 + 1, 1, sl, acc, true, true);
-        const int kkeys = nc >= 2 ? 8 : 4;       // K = keys present (16 per step)
-        for (int ks = 0; ks < kkeys; ++ks)
-          mma_ss(acc + 64, dsc(t_d, ds_a + ks * 2048),
-                 dsc(t_n, sl + kX + ks * 2048), idesc_nn, true);
+        if (nc > 1) bwd_issue_g(tmem, acc, sl, g0 + 1, 1, true, true);
+        if (nc >= 2) bwd_issue_r<8>(acc + 64, ds_lo, sl, true);
+        else bwd_issue_r<4>(acc + 64, ds_lo, sl, true);
         int nc_next = 0;
         uint32_t sl_next = 0;
         if (have_next) {
@@ -440,25 +451,28 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
             break;
           tc_fence_after();
           nc_next = min(3, n_chunks - 2 * nxt.p);
-          sl_next = slots_a + sn * kSlotBytes;
-          issue_s(n + 1, 0, nc_next, sl_next);
+          sl_next = slot0 + (uint32_t)(sn * kSlotBytes) / 16;
+          bwd_issue_s(tmem, sl_next, g0 + 3, 0, nc_next, &bar->s_full[(g0 + 3) & 1]);
         }
         // ---- block 2, then R1 = dS[block 2, zeros] X_K into the other set's dK
-        if (!wait_p(g0 + 2)) break;
+        if (!bwd_wait_p(bar, g0 + 2, abort, status)) break;
         tc_fence_after();
         if (nc == 3) {
-          issue_g(g0 + 2, 2, sl, acc, true, true);
-          if (!wait_acc(a ^ 1, (n + 1) >> 1)) break;
+          bwd_issue_g(tmem, acc, sl, g0 + 2, 2, true, true);
+          const int b = a ^ 1, need_b = (n + 1) >> 1;
+          int& seen_b = b ? seen1 : seen0;
+          while (ok && seen_b < need_b)
+            ok = mbar_wait(&bar->acc_free[b], (uint32_t)(seen_b++) & 1u, abort, status);
+          if (!ok) break;
           tc_fence_after();
-          const uint32_t acc2 = tmem + kColAcc + (uint32_t)(a ^ 1) * 128;
-          for (int ks = 0; ks < 8; ++ks)
-            mma_ss(acc2 + 64, dsc(t_d, ds_a + 2 * kDsBlock + ks * 2048),
-                   dsc(t_n, sl + kX + ks * 2048), idesc_nn, ks > 0);
+          bwd_issue_r<8>(tmem + kColAcc + (uint32_t)b * 128 + 64, ds_lo + 2 * (kDsBlock / 16), sl,
+                         false);
         }
         mma_commit(&bar->g_full[a]);
         mma_commit(&bar->slot_free[s]);
         prev_r1_alone = cur.last && nc == 3;
-        if (have_next) issue_s(n + 1, 1, nc_next, sl_next);
+        if (have_next)
+          bwd_issue_s(tmem, sl_next, g0 + 4, 1, nc_next, &bar->s_full[(g0 + 4) & 1]);
         cur = nxt;
         have = have_next;
         ++n;

@@ -145,6 +145,52 @@ __device__ __forceinline__ void convert_row(uint8_t* tile, int row, int half) {
   }
 }
 
+// ---- MMA issue helpers (one thread); descriptor lower words are shared
+// addresses >> 4 plus the LBO field of the operand layout.
+constexpr uint32_t kIdS64 = idesc_f16(128, 64, 1, false, false);    // Q K^T: bf16, K-major
+constexpr uint32_t kIdS128 = idesc_f16(128, 128, 1, false, false);
+constexpr uint32_t kIdO = idesc_f16(128, 64, 0, false, true);       // P V: fp16, V MN-major
+constexpr uint32_t kLboK = desc_lbo(16), kLboV = desc_lbo(kTile);
+
+// S = Q K^T of job nn (slot nn % kSlots, TMEM buffer nn & 1): key block 0 is
+// the previous chunk (side buffer pb, or the previous slot's odd chunk);
+// blocks 1 and 2 (this slot's chunks, contiguous) go in one N = 128 product.
+__device__ __forceinline__ bool fwd_issue_s(FwdBar* bar, uint32_t tmem, uint32_t slot0,
+                                            uint32_t pre0, const Job& jb, int nn, int pb,
+                                            int n_chunks, volatile int* abort, int* status) {
+  const int s = nn % kSlots, b = nn & 1;
+  if (!mbar_wait(&bar->slot_full[s], (uint32_t)(nn / kSlots) & 1u, abort, status)) return false;
+  tc_fence_after();
+  const uint32_t sl = slot0 + (uint32_t)(s * kSlotBytes) / 16;
+  const uint32_t d = tmem + (uint32_t)b * kSCols;
+  const bool has_prev = jb.p > 0, has_odd = 2 * jb.p + 1 < n_chunks;
+  const uint32_t q = sl + kLboK;
+  if (has_prev) {
+    const uint32_t prev_x = pb >= 0 ? pre0 + (uint32_t)(pb * kPreBytes) / 16
+                                    : slot0 + (uint32_t)(((nn + kSlots - 1) % kSlots) * kSlotBytes + kTile) / 16;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      mma_ss_w(d, q + 2 * ks, prev_x + kLboK + 2 * ks, kDescHi1024, kIdS64, ks > 0);
+  }
+  if (has_odd) {
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      mma_ss_w(d + 64, q + 2 * ks, q + 2 * ks, kDescHi1024, kIdS128, ks > 0);
+  } else {
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      mma_ss_w(d + 64, q + 2 * ks, q + 2 * ks, kDescHi1024, kIdS64, ks > 0);
+  }
+  mma_commit(&bar->s_full[b]);
+  return true;
+}
+// O (+)= P[:, 64 keys] V_block with P from TMEM.
+__device__ __forceinline__ void fwd_issue_pv(uint32_t d, uint32_t pa, uint32_t v_lo, bool acc) {
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks)
+    mma_ts_w(d, pa + ks * 8, v_lo + 128 * ks, kDescHi1024, kIdO, acc || ks > 0);
+}
+
 template <bool kCausal>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __restrict__ v,
@@ -284,48 +330,23 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
     // ------------------------------------------------ MMA issuer (warp 12)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
     if (warp == 12 && lane == 0) {
-      const uint32_t idesc_s = idesc_f16(128, 64, 1, false, false);   // Q K^T: bf16, K-major
-      const uint32_t idesc_o = idesc_f16(128, 64, 0, false, true);    // P V, V MN-major
-      const uint32_t slots_a = smem_u32(slots), pres_a = smem_u32(pres);
+      const uint32_t slot0 = smem_u32(slots) >> 4, pre0 = smem_u32(pres) >> 4;
       JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
       Job cur, nxt;
       bool have_cur = it.next(cur);
       int n = 0, pre_uses = 0;
       int cur_pre = -1, nxt_pre = -1;
       bool ok = true;
-      // S for job nn (slot nn % kSlots, TMEM buffer nn & 1)
-      auto issue_s = [&](const Job& jb, int nn, int pb) -> bool {
-        const int s = nn % kSlots, b = nn & 1;
-        if (!mbar_wait(&bar->slot_full[s], (uint32_t)(nn / kSlots) & 1u, abort, status)) return false;
-        tc_fence_after();
-        const uint32_t sl = slots_a + s * kSlotBytes;
-        const uint32_t d = tmem + (uint32_t)b * kSCols;
-        const bool has_prev = jb.p > 0, has_odd = 2 * jb.p + 1 < n_chunks;
-        const uint32_t prev_x = pb >= 0 ? pres_a + pb * kPreBytes
-                                        : slots_a + ((nn + kSlots - 1) % kSlots) * kSlotBytes + kTile;
-#pragma unroll
-        for (int kb = 0; kb < 3; ++kb) {
-          if ((kb == 0 && !has_prev) || (kb == 2 && !has_odd)) continue;
-          const uint32_t key = kb == 0 ? prev_x : (kb == 1 ? sl : sl + kTile);
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t a = smem_desc(sl + ks * 32, 16, 1024);
-            const uint64_t bd = smem_desc(key + ks * 32, 16, 1024);
-            mma_ss(d + kb * 64, a, bd, idesc_s, ks > 0 ? 1u : 0u);
-          }
-        }
-        mma_commit(&bar->s_full[b]);
-        return true;
-      };
       if (have_cur) {
         if (cur.first && cur.p > 0) cur_pre = pre_uses++ % kPre;
-        ok = issue_s(cur, 0, cur_pre);
+        ok = fwd_issue_s(bar, tmem, slot0, pre0, cur, 0, cur_pre, n_chunks, abort, status);
       }
       while (have_cur && ok) {
         const bool have_nxt = it.next(nxt);
         nxt_pre = -1;
         if (have_nxt && nxt.first && nxt.p > 0) nxt_pre = pre_uses++ % kPre;
-        if (have_nxt && !issue_s(nxt, n + 1, nxt_pre)) break;
+        if (have_nxt && !fwd_issue_s(bar, tmem, slot0, pre0, nxt, n + 1, nxt_pre, n_chunks, abort, status))
+          break;
         // O = P V for job n
         const int b = n & 1;
         if (!mbar_wait(&bar->p_full[b], (uint32_t)(n / 2) & 1u, abort, status)) break;
@@ -333,25 +354,17 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
           break;
         tc_fence_after();
         const int s = n % kSlots;
-        const uint32_t sl = slots_a + s * kSlotBytes;
+        const uint32_t sl = slot0 + (uint32_t)(s * kSlotBytes) / 16;
         const bool has_prev = cur.p > 0, has_odd = 2 * cur.p + 1 < n_chunks;
-        const uint32_t prev_v = cur_pre >= 0
-                                    ? pres_a + cur_pre * kPreBytes + kTile
-                                    : slots_a + ((n + kSlots - 1) % kSlots) * kSlotBytes + 3 * kTile;
+        const uint32_t prev_v =
+            cur_pre >= 0 ? pre0 + (uint32_t)(cur_pre * kPreBytes + kTile) / 16
+                         : slot0 + (uint32_t)(((n + kSlots - 1) % kSlots) * kSlotBytes + 3 * kTile) / 16;
         const uint32_t d = tmem + kOCol + (uint32_t)b * 64;
         const uint32_t pa = tmem + (uint32_t)b * kSCols;
-        bool acc = false;
-#pragma unroll
-        for (int kb = 0; kb < 3; ++kb) {
-          if ((kb == 0 && !has_prev) || (kb == 2 && !has_odd)) continue;
-          const uint32_t val = kb == 0 ? prev_v : (kb == 1 ? sl + 2 * kTile : sl + 3 * kTile);
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t bd = smem_desc(val + ks * 2048, 8192, 1024);
-            mma_ts(d, pa + kb * 32 + ks * 8, bd, idesc_o, acc ? 1u : 0u);
-            acc = true;
-          }
-        }
+        // key block 0 (previous chunk) when present, then blocks 1 and 2
+        if (has_prev) fwd_issue_pv(d, pa, prev_v + kLboV, false);
+        fwd_issue_pv(d, pa + 32, sl + 2 * kTile / 16 + kLboV, has_prev);
+        if (has_odd) fwd_issue_pv(d, pa + 64, sl + 3 * kTile / 16 + kLboV, true);
         mma_commit(&bar->p_free[b]);                    // P(n) consumed, O(n) ready
         if (n >= 1) mma_commit(&bar->slot_free[(n - 1) % kSlots]);
         if (cur_pre >= 0) mma_commit(&bar->pre_free[cur_pre]);

@@ -147,33 +147,10 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
       // the chunks of a pair of tiles are interleaved so both stay busy.
       if (mbar_wait(&bar->r_full, 0, abort, status)) {
         tc_fence_after();
-        const uint32_t r_base = smem_u32(r_smem);
-        const uint32_t x_base = smem_u32(x_smem);
-        int uses[2] = {0, 0};
+        const uint32_t r_lo = (smem_u32(r_smem) >> 4) | desc_lbo(kRBlockBytes);
+        const uint32_t x_lo = (smem_u32(x_smem) >> 4) | desc_lbo(16);
+        int uses0 = 0, uses1 = 0;
         bool ok = true;
-        auto issue = [&](int it, int j) -> bool {
-          const int w = it & 1, s = it % kStages;
-          if (uses[w] > 0 &&
-              !mbar_wait(&bar->acc_empty[w], (uint32_t)(uses[w] - 1) & 1u, abort, status))
-            return false;
-          ++uses[w];
-          tc_fence_after();
-          const int ncols = min(kChunkN, nh - j * kChunkN);
-          // whole 64-column blocks: the MN-major operand is read in complete
-          // swizzle atoms; the zero-filled extra columns are masked later
-          const int n_mma = (ncols + 63) / 64 * 64;
-          const uint32_t idesc = idesc_f16(kTileM, n_mma, 1, false, true);
-          const uint32_t d = tmem + (uint32_t)(w * kChunkN);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            uint64_t a = smem_desc(x_base + s * kXBytes + k * 32, 16, 1024);
-            uint64_t b = smem_desc(r_base + j * 4 * kRBlockBytes + k * 2048, kRBlockBytes, 1024);
-            mma_ss(d, a, b, idesc, k > 0 ? 1u : 0u);
-          }
-          mma_commit(&bar->acc_full[w]);
-          if (j == nsub - 1) mma_commit(&bar->x_empty[s]);
-          return true;
-        };
         const int n_mine = (n_tiles - ci + ctas_per_round - 1) / ctas_per_round;
         for (int it0 = 0; it0 < n_mine && ok; it0 += 2) {
           const int cnt = min(2, n_mine - it0);
@@ -183,7 +160,30 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
           if (!ok) break;
           tc_fence_after();
           for (int j = 0; j < nsub && ok; ++j)
-            for (int k = 0; k < cnt && ok; ++k) ok = issue(it0 + k, j);
+            for (int k = 0; k < cnt && ok; ++k) {
+              const int it = it0 + k, w = it & 1, s = it % kStages;
+              int& uses = w ? uses1 : uses0;
+              if (uses > 0 &&
+                  !mbar_wait(&bar->acc_empty[w], (uint32_t)(uses - 1) & 1u, abort, status)) {
+                ok = false;
+                break;
+              }
+              ++uses;
+              tc_fence_after();
+              const int ncols = min(kChunkN, nh - j * kChunkN);
+              // whole 64-column blocks: the MN-major operand is read in complete
+              // swizzle atoms; the zero-filled extra columns are masked later
+              const int n_mma = (ncols + 63) / 64 * 64;
+              const uint32_t idesc = idesc_f16(kTileM, n_mma, 1, false, true);
+              const uint32_t d = tmem + (uint32_t)(w * kChunkN);
+              const uint32_t a = x_lo + (uint32_t)(s * kXBytes) / 16;
+              const uint32_t b = r_lo + (uint32_t)(j * 4 * kRBlockBytes) / 16;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_ss_w(d, a + 2 * kk, b + 128 * kk, kDescHi1024, idesc, kk > 0);
+              mma_commit(&bar->acc_full[w]);
+              if (j == nsub - 1) mma_commit(&bar->x_empty[s]);
+            }
         }
       }
       // all issued MMAs have finished before TMEM is released (bounded)
