@@ -22,8 +22,17 @@
 namespace lsh {
 namespace tc {
 
-// Bounded spin: polls before a wait is declared timed out (about a second).
-constexpr uint32_t kSpinLimit = 1u << 24;
+// Bounded waits: a waiting thread is suspended in the barrier for up to
+// kSuspendNs per poll (woken as soon as the phase completes), so waiting warps
+// take no issue slots from working ones; after kWaitLimitNs of global time
+// (one second) the wait is declared timed out.
+constexpr uint32_t kSuspendNs = 1000;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -47,17 +56,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The same poll, allowing the thread to be suspended for up to kSuspendNs.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
 // Waits for the phase with the given parity to complete. Gives up after
-// kSpinLimit polls, or as soon as *abort is set by another thread; on a
-// timeout it records LSH_ERR_TIMEOUT and sets *abort. Returns false if it
-// gave up.
+// kWaitLimitNs, or as soon as *abort is set by another thread; on a timeout it
+// records LSH_ERR_TIMEOUT and sets *abort. Returns false if it gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 63) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_suspend(bar, parity)) return true;
+    if ((i & 7) == 0) {
       if (*abort) return false;
-      if (i > 4096) __nanosleep(32);
+      if (global_ns() - t0 > kWaitLimitNs) break;
     }
   }
   if (status) atomicExch(status, (int)LSH_ERR_TIMEOUT);
