@@ -12,7 +12,8 @@
 // segment — 128 keys, one per TMEM lane. The queries that see them are
 // chunks 2p, 2p+1, 2p+2 (chunk c sees chunks c-1 and c): three query blocks
 // of 64; key rows of chunk 2p see blocks 0-1, rows of chunk 2p+1 blocks 1-2.
-// Each block is one pipeline step:
+// Each block is one pipeline step, in the order 1, 0, 2 (the block that all
+// 128 key rows see, whose softmax is the longest, goes first):
 //   S^T = X_K X_qb^T, dP^T = V_K dO_qb^T        (M=128 keys, N=64)
 //   P^T and dS^T (fp16, in place over S^T and dP^T in TMEM; dS^T also to
 //   shared memory for the query-side products)
@@ -405,8 +406,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
         if (ok) {
           tc_fence_after();
           const int nc = min(3, n_chunks - 2 * cur.p);
-          bwd_issue_s(tmem, slot0, 0, 0, nc, &bar->s_full[0]);
-          bwd_issue_s(tmem, slot0, 1, 1, nc, &bar->s_full[1]);
+          bwd_issue_s(tmem, slot0, 0, 1, nc, &bar->s_full[0]);
+          bwd_issue_s(tmem, slot0, 1, 0, nc, &bar->s_full[1]);
         }
       }
       int n = 0;
@@ -418,7 +419,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
         const uint32_t sl = slot0 + (uint32_t)(s * kSlotBytes) / 16;
         const uint32_t acc = tmem + kColAcc + (uint32_t)a * 128;
         const int g0 = 3 * n;
-        // ---- block 0 (always present)
+        // ---- step 0: query block 1 (the one all 128 key rows see)
         if (!bwd_wait_p(bar, g0, abort, status)) break;
         // flushes of the earlier items that used set a (and, after a unit's
         // last item, of that item too: it read its R1 rows from set a)
@@ -435,12 +436,12 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
           if (!ok) break;
         }
         tc_fence_after();
-        bwd_issue_g(tmem, acc, sl, g0, 0, false, !cur.first);
+        if (nc > 1) bwd_issue_g(tmem, acc, sl, g0, 1, false, !cur.first);
         bwd_issue_s(tmem, sl, g0 + 2, 2, nc, &bar->s_full[(g0 + 2) & 1]);
-        // ---- block 1, then R0 = dS[blocks 0,1] X_K into dK
+        // ---- step 1: query block 0, then R0 = dS[blocks 0,1] X_K into dK
         if (!bwd_wait_p(bar, g0 + 1, abort, status)) break;
         tc_fence_after();
-        if (nc > 1) bwd_issue_g(tmem, acc, sl, g0 + 1, 1, true, true);
+        bwd_issue_g(tmem, acc, sl, g0 + 1, 0, nc > 1, nc > 1 || !cur.first);
         if (nc >= 2) bwd_issue_r<8>(acc + 64, ds_lo, sl, true);
         else bwd_issue_r<4>(acc + 64, ds_lo, sl, true);
         int nc_next = 0;
@@ -452,9 +453,9 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
           tc_fence_after();
           nc_next = min(3, n_chunks - 2 * nxt.p);
           sl_next = slot0 + (uint32_t)(sn * kSlotBytes) / 16;
-          bwd_issue_s(tmem, sl_next, g0 + 3, 0, nc_next, &bar->s_full[(g0 + 3) & 1]);
+          bwd_issue_s(tmem, sl_next, g0 + 3, 1, nc_next, &bar->s_full[(g0 + 3) & 1]);
         }
-        // ---- block 2, then R1 = dS[block 2, zeros] X_K into the other set's dK
+        // ---- step 2: query block 2, then R1 = dS[block 2, zeros] X_K into the other set's dK
         if (!bwd_wait_p(bar, g0 + 2, abort, status)) break;
         tc_fence_after();
         if (nc == 3) {
@@ -472,7 +473,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
         mma_commit(&bar->slot_free[s]);
         prev_r1_alone = cur.last && nc == 3;
         if (have_next)
-          bwd_issue_s(tmem, sl_next, g0 + 4, 1, nc_next, &bar->s_full[(g0 + 4) & 1]);
+          bwd_issue_s(tmem, sl_next, g0 + 4, 0, nc_next, &bar->s_full[(g0 + 4) & 1]);
         cur = nxt;
         have = have_next;
         ++n;
@@ -545,8 +546,10 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
     while (ok && it.next(j)) {
       const int s = n % kSlots;
       const int nc = min(3, n_chunks - 2 * j.p);
-      for (int qb = 0; qb < 3; ++qb) {
-        if (((3 * n + qb) & 1) != w) continue;
+      for (int kstep = 0; kstep < 3; ++kstep) {
+        // steps of an item take query blocks 1, 0, 2 (the full block first)
+        const int qb = kstep == 0 ? 1 : (kstep == 1 ? 0 : 2);
+        if (((3 * n + kstep) & 1) != w) continue;
         if (!warp_ok(mbar_wait(&bar->s_full[w], (uint32_t)k & 1u, abort, status))) {
           ok = false;
           break;
