@@ -30,8 +30,9 @@
 //                one query row per thread, two passes over its S row in TMEM:
 //                (1) causal/self mask and row max, masked values written back;
 //                (2) exp2, row sum, P packed as fp16 pairs into TMEM over S.
-//                The warpgroup then writes its previous job's output: O from
-//                TMEM scaled by 1/l, as fp16, in original token order, + lse_r.
+//                After publishing P, the warpgroup writes its previous job's
+//                output: O from TMEM scaled by 1/l, as fp16, in original token
+//                order, + lse_r (so the stores stay off the path from S to P).
 // fp16 for P and V keeps P's rounding error at 2^-11 (bf16 would add about
 // 3e-3 to O on the 64K workload).
 #include <cuda_fp16.h>
@@ -430,8 +431,6 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
       const bool use_pre = j.first && j.p > 0;
       const int pb = use_pre ? pre_uses++ % kPre : -1;
       if ((n & 1) != wg) { ++n; continue; }
-      if (pend && !epilogue()) break;
-      pend = false;
       const int s = n % kSlots;
       if (!mbar_wait(&bar->s_full[wg], (uint32_t)(n / 2) & 1u, abort, status)) break;
       tc_fence_after();
@@ -508,6 +507,9 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bar->p_full[wg]);
+      // the previous job's output is written now, off the path from S to P
+      // (this job's PV waits only for its TMEM read, signalled by o_free)
+      if (pend && !epilogue()) break;
       pend = true;
       pend_n = n;
       pend_write = row_live;
