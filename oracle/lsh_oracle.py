@@ -20,7 +20,7 @@ What it computes, step by step, in the order of the source pages:
 * Same page, Key points, "Number of hash rounds": several rounds, each an
   independent hash.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   scale = 1/sqrt(d) on the logits; argmax ties go to the lowest index; the
   sort is stable by position; the window is the chunk and the previous chunk
   of the same round, with no wrap-around; causal masking is by original
