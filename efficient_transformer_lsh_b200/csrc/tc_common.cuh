@@ -252,31 +252,14 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int ab_type, bool
          | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// D[tmem] (+)= A[smem] * B[smem]; issued by one thread.
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// D[tmem] (+)= A[tmem] * B[smem]: A is M x K in TMEM (lane = row, two 16-bit
-// elements per 32-bit column, the lower K index in the low half).
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// The same two MMAs with each shared-memory descriptor given as its two 32-bit
-// words: lo = (address >> 4) | (LBO >> 4) << 16, hi = the SBO / version /
-// swizzle word. Issuers keep per-tile `lo` words and add constant offsets
-// (bytes / 16; addresses stay below 256 KB, so no carry leaves the field).
+// D[tmem] (+)= A * B, issued by one thread, with each shared-memory
+// descriptor given as its two 32-bit words: lo = (address >> 4) | (LBO >> 4)
+// << 16, hi = the SBO / version / swizzle word (smem_desc's upper half).
+// Issuers keep per-tile `lo` words and add constant offsets (bytes / 16;
+// addresses stay below 256 KB, so no carry leaves the field).
+// mma_ss_w: A and B in shared memory. mma_ts_w: A in TMEM (M x K, lane =
+// row, two 16-bit elements per 32-bit column, the lower K index in the low
+// half), B in shared memory.
 __device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
                                          uint32_t hi, uint32_t idesc, uint32_t accumulate) {
   asm volatile(
