@@ -18,14 +18,14 @@
 //   P^T and dS^T (fp16, in place over S^T and dP^T in TMEM; dS^T also to
 //   shared memory for the query-side products)
 //   dV += P^T dO_qb,  dK += dS^T X_qb           (A from TMEM, accumulated in TMEM)
-// and after blocks 0-1 / block 2 the query-side terms through the
+// and once blocks 1 and 0 / block 2 are done, the query-side terms through the
 // transposed (MN-major) reading of the dS^T tiles:
 //   R0 = dS[blocks 0,1] X_K — for chunks 2p, 2p+1, i.e. the same tokens as
 //        the key rows, lane for lane: accumulated straight into dK;
 //   R1 = dS[block 2, zeros] X_K — for chunk 2p+2, which is the first key
 //        chunk of the next pair: written into the OTHER accumulator set's dK,
 //        so that the next item of the same unit adds its own terms on top.
-//        At the end of a unit it is flushed on its own.
+//        At the end of a unit it is stored on its own (the edge rows below).
 // The finished rows dV and scale*dK of an item are stored, converted to fp16,
 // as per-round partial gradients in sorted (slot) order — 128 consecutive
 // rows, two TMA tile stores per tensor; unit-end R1 rows go to a small edge
