@@ -587,7 +587,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
                   const bool valid = kCausal ? (kpos < qq[e]) : (kpos != qq[e]);
                   const float pr = ex2(fmaf(__uint_as_float(sv[i]), scale_log2, -ll[e]));
                   pe[e] = valid ? pr : 0.f;
-                  de[e] = valid ? pr * (__uint_as_float(pv[i]) - dd[e]) : 0.f;
+                  // pe is 0 where masked and dP - D is finite, so no second select
+                  de[e] = pe[e] * (__uint_as_float(pv[i]) - dd[e]);
                 }
                 pk[2 * i4] = pack_f16x2(pe[0], pe[1]);
                 pk[2 * i4 + 1] = pack_f16x2(pe[2], pe[3]);
