@@ -24,9 +24,13 @@
  *   - Arguments are checked on the host before anything is launched; a bad
  *     argument returns LSH_ERR_INVALID_ARG / LSH_ERR_UNSUPPORTED /
  *     LSH_ERR_WORKSPACE and launches nothing. A failed launch returns
- *     LSH_ERR_CUDA. Kernels that wait on hardware barriers give up after a
- *     bounded number of polls and record LSH_ERR_TIMEOUT in a device status
- *     word, read by lsh_device_status(). No C++ exception crosses the ABI.
+ *     LSH_ERR_CUDA. Kernels that wait on hardware barriers give up after one
+ *     second of waiting and record LSH_ERR_TIMEOUT in a device status word,
+ *     read by lsh_device_status(). No C++ exception crosses the ABI.
+ *   - bf16 problems with chunk 64 run on the tensor cores, where gathered
+ *     rows, attention weights and their gradients pass through fp16 (fp32
+ *     accumulation): inputs, outputs and gradients must stay inside the fp16
+ *     range (|value| < 65504). Other problems run on CUDA cores in fp32.
  *   - Outputs are overwritten, never accumulated into.
  *   - Shapes: B batch, H heads, L sequence length, d head size (64),
  *     n_buckets (even), n_rounds hash rounds, chunk = m.
