@@ -342,3 +342,85 @@ def lsh_attention(qk, v, R, m, causal, scale):
     perm = sort_positions(bucket)
     O, LSE = forward(qk, v, perm, m, causal, scale)
     return {"bucket": bucket, "gap": gap, "perm": perm, "O": O, "LSE": LSE}
+
+
+# --------------------------------------------------------------------------
+# Local chunked self-attention ("The Reformer – Pushing the limits of
+# language modeling", Approach and Takeaways: the input is cut into chunks of
+# length l_c, and each chunk also sees a configurable overlap of preceding
+# and following chunks). Readings where the page is silent: the overlap is a
+# whole number of chunks (n_back before, n_fwd after, clipped at the sequence
+# ends); queries and keys are the shared qk vectors with the same self-mask
+# and fall-back as the LSH layer, and causal masking is by position.
+# --------------------------------------------------------------------------
+
+def local_window(c: int, m: int, L: int, n_back: int, n_fwd: int) -> range:
+    """Key positions seen by the queries of chunk ``c``."""
+    return range(max(0, (c - n_back) * m), min(L, (c + 1 + n_fwd) * m))
+
+
+def local_forward(qk, v, m, n_back, n_fwd, causal, scale):
+    """Local attention forward: (O [B,H,L,d], LSE [B,H,L]).
+
+    Chunk c's queries (positions [cm, (c+1)m)) attend to the keys of
+    ``local_window``; a query with no valid key attends to itself (O = v,
+    LSE = -inf).
+    """
+    qk = np.asarray(qk, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, H, L, d = qk.shape
+    if L % m:
+        raise ValueError("L must be a multiple of the chunk size")
+    O = np.zeros_like(v)
+    LSE = np.full((B, H, L), NEG_INF)
+    for b in range(B):
+        for h in range(H):
+            X, V = qk[b, h], v[b, h]
+            for c in range(L // m):
+                qi = np.arange(c * m, (c + 1) * m)
+                kj = np.array(local_window(c, m, L, n_back, n_fwd))
+                s = scale * (X[qi] @ X[kj].T)
+                valid = _valid(qi, kj, causal)
+                lse = _masked_lse(s, valid)
+                fin = np.isfinite(lse)
+                with np.errstate(under="ignore"):
+                    w = np.where(valid & fin[:, None],
+                                 np.exp(s - np.where(fin, lse, 0.0)[:, None]), 0.0)
+                O[b, h, qi] = np.where(fin[:, None], w @ V[kj], V[qi])
+                LSE[b, h, qi] = lse
+    return O, LSE
+
+
+def local_backward(qk, v, m, n_back, n_fwd, causal, scale, O, LSE, dO):
+    """Gradients of sum(O * dO) for local attention, by recomputation.
+
+    Same algebra as ``backward`` with the local windows: P = exp(s - LSE),
+    dS = P (dO_i . v_j - D_i), both query- and key-side terms into dqk, and
+    rows that fell back to themselves pass dO to dv.
+    """
+    qk = np.asarray(qk, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    dO = np.asarray(dO, dtype=np.float64)
+    B, H, L, d = qk.shape
+    dqk = np.zeros_like(qk)
+    dv = np.zeros_like(v)
+    D = (dO * np.asarray(O, dtype=np.float64)).sum(axis=-1)
+    for b in range(B):
+        for h in range(H):
+            X, V, G = qk[b, h], v[b, h], dO[b, h]
+            for c in range(L // m):
+                qi = np.arange(c * m, (c + 1) * m)
+                kj = np.array(local_window(c, m, L, n_back, n_fwd))
+                s = scale * (X[qi] @ X[kj].T)
+                lq = LSE[b, h, qi]
+                fin = np.isfinite(lq)
+                valid = _valid(qi, kj, causal) & fin[:, None]
+                with np.errstate(under="ignore"):
+                    P = np.where(valid, np.exp(s - np.where(fin, lq, 0.0)[:, None]), 0.0)
+                dS = P * (G[qi] @ V[kj].T - D[b, h, qi][:, None])
+                dqk[b, h, qi] += scale * (dS @ X[kj])
+                dqk[b, h, kj] += scale * (dS.T @ X[qi])
+                dv[b, h, kj] += P.T @ G[qi]
+            fb = ~np.isfinite(LSE[b, h])
+            dv[b, h, fb] += G[fb]
+    return dqk, dv
