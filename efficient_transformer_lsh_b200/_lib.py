@@ -16,12 +16,14 @@ LIB_PATH = os.path.join(PKG, "liblsh.so")
 LSH_F32, LSH_BF16 = 0, 1
 STATUS_NAMES = {
     0: "LSH_OK", 1: "LSH_ERR_INVALID_ARG", 2: "LSH_ERR_UNSUPPORTED", 3: "LSH_ERR_WORKSPACE",
-    4: "LSH_ERR_CUDA", 5: "LSH_ERR_TIMEOUT", 6: "LSH_ERR_DEVICE_CHECK",
+    4: "LSH_ERR_CUDA", 5: "LSH_ERR_TIMEOUT", 6: "LSH_ERR_DEVICE_CHECK", 7: "LSH_ERR_RANGE",
 }
 # Every symbol include/lsh.h declares.
 EXPORTS = ("lsh_hash", "lsh_sort_workspace_size", "lsh_sort", "lsh_fwd_workspace_size",
            "lsh_attn_fwd", "lsh_bwd_workspace_size", "lsh_attn_bwd", "lsh_device_status",
-           "lsh_status_string", "lsh_launch_count", "lsh_sort_noalloc")
+           "lsh_status_string", "lsh_launch_count", "lsh_sort_noalloc", "lsh_check_wait_timeout",
+           "lsh_local_fwd_workspace_size", "lsh_local_attn_fwd", "lsh_local_bwd_workspace_size",
+           "lsh_local_attn_bwd")
 # Size of the library-owned scratch used by lsh_sort_noalloc (matches lsh.h).
 SORT_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -61,7 +63,7 @@ def lib() -> ctypes.CDLL:
                 f"{LIB_PATH} is missing: build it with `python -m efficient_transformer_lsh_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
         P = ctypes.POINTER(lsh_problem)
-        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
         sig = {
             "lsh_hash": ([P, vp, vp, vp, vp], ctypes.c_int),
             "lsh_sort_workspace_size": ([P], sz),
@@ -74,6 +76,12 @@ def lib() -> ctypes.CDLL:
             "lsh_status_string": ([ctypes.c_int], ctypes.c_char_p),
             "lsh_launch_count": ([], ctypes.c_uint64),
             "lsh_sort_noalloc": ([P, vp, vp, vp], ctypes.c_int),
+            "lsh_check_wait_timeout": ([ctypes.c_uint64, vp], ctypes.c_int),
+            "lsh_local_fwd_workspace_size": ([P, i32, i32], sz),
+            "lsh_local_attn_fwd": ([P, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+            "lsh_local_bwd_workspace_size": ([P, i32, i32], sz),
+            "lsh_local_attn_bwd": ([P, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+                                   ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -150,8 +158,37 @@ def lsh_attn_bwd(p: lsh_problem, qk, v, perm, out, out_lo, lse, dout, dqk, dv, w
                               int(ws_bytes), _stream(stream)), "lsh_attn_bwd")
 
 
+def lsh_local_fwd_workspace_size(p: lsh_problem, n_back: int, n_fwd: int) -> int:
+    return int(lib().lsh_local_fwd_workspace_size(ctypes.byref(p), int(n_back), int(n_fwd)))
+
+
+def lsh_local_attn_fwd(p: lsh_problem, n_back, n_fwd, qk, v, out, out_lo, lse, ws, ws_bytes: int,
+                       stream=None):
+    _check(lib().lsh_local_attn_fwd(ctypes.byref(p), int(n_back), int(n_fwd), _ptr(qk), _ptr(v),
+                                    _ptr(out), _ptr(out_lo), _ptr(lse), _ptr(ws), int(ws_bytes),
+                                    _stream(stream)), "lsh_local_attn_fwd")
+
+
+def lsh_local_bwd_workspace_size(p: lsh_problem, n_back: int, n_fwd: int) -> int:
+    return int(lib().lsh_local_bwd_workspace_size(ctypes.byref(p), int(n_back), int(n_fwd)))
+
+
+def lsh_local_attn_bwd(p: lsh_problem, n_back, n_fwd, qk, v, out, out_lo, lse, dout, dqk, dv, ws,
+                       ws_bytes: int, stream=None):
+    _check(lib().lsh_local_attn_bwd(ctypes.byref(p), int(n_back), int(n_fwd), _ptr(qk), _ptr(v),
+                                    _ptr(out), _ptr(out_lo), _ptr(lse), _ptr(dout), _ptr(dqk),
+                                    _ptr(dv), _ptr(ws), int(ws_bytes), _stream(stream)),
+           "lsh_local_attn_bwd")
+
+
 def lsh_device_status(stream=None) -> int:
     return int(lib().lsh_device_status(_stream(stream)))
+
+
+def lsh_check_wait_timeout(limit_ns: int, stream=None):
+    """Runs the bounded-wait failure path once (see lsh.h); read the result
+    with lsh_device_status()."""
+    _check(lib().lsh_check_wait_timeout(int(limit_ns), _stream(stream)), "lsh_check_wait_timeout")
 
 
 def lsh_launch_count() -> int:

@@ -10,6 +10,12 @@ namespace lsh {
 
 constexpr int kD = 64;  // head size supported by every kernel
 
+// Records an error code in the device status word unless one is already
+// there: the first error of a sequence of launches is the one reported.
+__device__ __forceinline__ void record_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
 // Widen 4 consecutive elements to float.
 __device__ __forceinline__ float4 load4(const float* p) {
   return *reinterpret_cast<const float4*>(p);

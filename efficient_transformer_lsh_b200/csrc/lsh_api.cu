@@ -5,9 +5,25 @@
 #include <mutex>
 
 #include "internal.h"
+#include "tc_common.cuh"
 
 namespace lsh {
 namespace {
+
+// One thread waits, through the bounded wait of the tensor-core pipelines, on
+// a barrier that nothing arrives on; the wait runs out after limit_ns and
+// records LSH_ERR_TIMEOUT. No asynchronous copy or MMA is in flight.
+__global__ void wait_timeout_kernel(uint64_t limit_ns, int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bar, 1);
+    abort = 0;
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) tc::mbar_wait(&bar, 0u, (volatile int*)&abort, status, limit_ns);
+}
 
 std::atomic<uint64_t> g_launches{0};
 
@@ -140,6 +156,58 @@ lsh_status lsh_attn_bwd(const lsh_problem* p, const void* qk, const void* v, con
                                      device_status_word(), (cudaStream_t)stream));
 }
 
+static lsh_status check_local(const lsh_problem* p, int32_t n_back, int32_t n_fwd) {
+  lsh_status st = check_problem(p);
+  if (st != LSH_OK) return st;
+  if (p->n_rounds != 1 || n_back < 0 || n_fwd < 0 || n_back > 65536 || n_fwd > 65536)
+    return LSH_ERR_INVALID_ARG;
+  return LSH_OK;
+}
+
+size_t lsh_local_fwd_workspace_size(const lsh_problem* p, int32_t n_back, int32_t n_fwd) {
+  if (check_local(p, n_back, n_fwd) != LSH_OK) return 0;
+  return local_fwd_ws_bytes(*p, n_back, n_fwd);
+}
+
+lsh_status lsh_local_attn_fwd(const lsh_problem* p, int32_t n_back, int32_t n_fwd, const void* qk,
+                              const void* v, void* out, void* out_lo, float* lse, void* ws,
+                              size_t ws_bytes, lsh_stream_t stream) {
+  lsh_status st = check_local(p, n_back, n_fwd);
+  if (st != LSH_OK) return st;
+  if (empty(p)) return LSH_OK;
+  if (!qk || !v || !out || !lse) return LSH_ERR_INVALID_ARG;
+  if (!aligned(qk, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(out_lo, 16))
+    return LSH_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < local_fwd_ws_bytes(*p, n_back, n_fwd) || !aligned(ws, 256))
+    return LSH_ERR_WORKSPACE;
+  if (p->dtype == LSH_F32) out_lo = nullptr;
+  return cuda_status(launch_local_fwd(*p, n_back, n_fwd, qk, v, out, out_lo, lse, ws,
+                                      device_status_word(), (cudaStream_t)stream));
+}
+
+size_t lsh_local_bwd_workspace_size(const lsh_problem* p, int32_t n_back, int32_t n_fwd) {
+  if (check_local(p, n_back, n_fwd) != LSH_OK) return 0;
+  return local_bwd_ws_bytes(*p, n_back, n_fwd);
+}
+
+lsh_status lsh_local_attn_bwd(const lsh_problem* p, int32_t n_back, int32_t n_fwd, const void* qk,
+                              const void* v, const void* out, const void* out_lo, const float* lse,
+                              const void* dout, float* dqk, float* dv, void* ws, size_t ws_bytes,
+                              lsh_stream_t stream) {
+  lsh_status st = check_local(p, n_back, n_fwd);
+  if (st != LSH_OK) return st;
+  if (empty(p)) return LSH_OK;
+  if (!qk || !v || !out || !lse || !dout || !dqk || !dv) return LSH_ERR_INVALID_ARG;
+  if (!aligned(qk, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(dout, 16) ||
+      !aligned(dqk, 16) || !aligned(dv, 16) || !aligned(out_lo, 16))
+    return LSH_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < local_bwd_ws_bytes(*p, n_back, n_fwd) || !aligned(ws, 256))
+    return LSH_ERR_WORKSPACE;
+  if (p->dtype == LSH_F32) out_lo = nullptr;
+  return cuda_status(launch_local_bwd(*p, n_back, n_fwd, qk, v, out, out_lo, lse, dout, dqk, dv,
+                                      ws, device_status_word(), (cudaStream_t)stream));
+}
+
 lsh_status lsh_device_status(lsh_stream_t stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return LSH_ERR_CUDA;
   int* w = device_status_word();
@@ -153,6 +221,15 @@ lsh_status lsh_device_status(lsh_stream_t stream) {
   return (lsh_status)v;
 }
 
+lsh_status lsh_check_wait_timeout(uint64_t limit_ns, lsh_stream_t stream) {
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return LSH_ERR_INVALID_ARG;
+  int* status = device_status_word();
+  if (!status) return LSH_ERR_CUDA;
+  wait_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(limit_ns, status);
+  note_launch();
+  return cuda_status(cudaGetLastError());
+}
+
 const char* lsh_status_string(lsh_status s) {
   switch (s) {
     case LSH_OK: return "ok";
@@ -162,6 +239,7 @@ const char* lsh_status_string(lsh_status s) {
     case LSH_ERR_CUDA: return "CUDA runtime error";
     case LSH_ERR_TIMEOUT: return "a kernel timed out waiting on a barrier";
     case LSH_ERR_DEVICE_CHECK: return "a kernel found an out-of-range index";
+    case LSH_ERR_RANGE: return "a tensor-core-path result is not finite (a value left the fp16 range)";
   }
   return "unknown status";
 }

@@ -16,9 +16,13 @@
  *
  * Conventions shared by every entry point
  *   - All tensor arguments are DEVICE pointers, contiguous, row-major, owned
- *     and allocated by the caller. The library allocates no memory; scratch
- *     space comes from the caller through (ws, ws_bytes), 256-byte aligned,
- *     of at least the size the matching *_workspace_size() returns.
+ *     and allocated by the caller. The library allocates no memory while it
+ *     runs: scratch space comes from the caller through (ws, ws_bytes),
+ *     256-byte aligned, of at least the size the matching *_workspace_size()
+ *     returns. Its only device memory is static, held by every GPU that loads
+ *     the library until the process exits: a 4-byte status word and the
+ *     16 MiB scratch array of lsh_sort_noalloc, whose contents persist from
+ *     one lsh_sort_noalloc call to the next.
  *   - Work is queued asynchronously on `stream` (NULL = legacy default
  *     stream). Nothing synchronises unless stated.
  *   - Arguments are checked on the host before anything is launched; a bad
@@ -30,7 +34,11 @@
  *   - bf16 problems with chunk 64 run on the tensor cores, where gathered
  *     rows, attention weights and their gradients pass through fp16 (fp32
  *     accumulation): inputs, outputs and gradients must stay inside the fp16
- *     range (|value| < 65504). Other problems run on CUDA cores in fp32.
+ *     range (|value| < 65504). This path checks every result it writes
+ *     (out, dqk, dv) and records LSH_ERR_RANGE in the device status word when
+ *     one is not finite, which is what an input or intermediate outside the
+ *     fp16 range produces; such a problem can be run on the CUDA cores by
+ *     passing float32 inputs. Other problems run on CUDA cores in fp32.
  *   - Outputs are overwritten, never accumulated into.
  *   - Shapes: B batch, H heads, L sequence length, d head size (64),
  *     n_buckets (even), n_rounds hash rounds, chunk = m.
@@ -60,7 +68,9 @@ typedef enum {
   LSH_ERR_WORKSPACE = 3,     /* workspace missing, too small or misaligned     */
   LSH_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed           */
   LSH_ERR_TIMEOUT = 5,       /* a kernel gave up waiting on a barrier          */
-  LSH_ERR_DEVICE_CHECK = 6   /* a kernel found an out-of-range index           */
+  LSH_ERR_DEVICE_CHECK = 6,  /* a kernel found an out-of-range index           */
+  LSH_ERR_RANGE = 7          /* a tensor-core-path result is not finite: an input
+                                or intermediate left the fp16 range            */
 } lsh_status;
 
 typedef enum { LSH_F32 = 0, LSH_BF16 = 1 } lsh_dtype;
@@ -138,6 +148,35 @@ lsh_status lsh_attn_bwd(const lsh_problem* p, const void* qk, const void* v,
                         void* ws, size_t ws_bytes, lsh_stream_t stream);
 
 /*
+ * lsh_local_attn_fwd / lsh_local_attn_bwd — local chunked self-attention
+ *   ("The Reformer - Pushing the limits of language modeling", Approach and
+ *   Takeaways: the input is cut into chunks of length l_c, and each chunk
+ *   also sees a configurable overlap of preceding and following chunks).
+ *   The queries of chunk c (positions [c m, (c+1) m)) attend to the keys at
+ *   positions [max(0, (c - n_back) m), min(L, (c + 1 + n_fwd) m)), with the
+ *   same shared-QK self-mask and fall-back, causal mask (j < i) and logit
+ *   scale as lsh_attn_fwd, i.e. lsh_attn_fwd's arithmetic in the identity
+ *   order with a window of n_back chunks before and n_fwd after.
+ *   - p->n_rounds must be 1; p->n_buckets is not used (any valid value).
+ *   - 0 <= n_back, n_fwd <= 65536, else LSH_ERR_INVALID_ARG.
+ *   - Outputs, out_lo and the backward's gradients as for lsh_attn_fwd /
+ *     lsh_attn_bwd; the workspaces come from the *_workspace_size calls with
+ *     the same (p, n_back, n_fwd).
+ *   - bf16 problems with chunk 64, n_back = 1 and n_fwd = 0 run on the tensor
+ *     cores (same fp16 range rule and LSH_ERR_RANGE check as the LSH path);
+ *     other problems run on CUDA cores in fp32.
+ */
+size_t lsh_local_fwd_workspace_size(const lsh_problem* p, int32_t n_back, int32_t n_fwd);
+lsh_status lsh_local_attn_fwd(const lsh_problem* p, int32_t n_back, int32_t n_fwd, const void* qk,
+                              const void* v, void* out, void* out_lo, float* lse, void* ws,
+                              size_t ws_bytes, lsh_stream_t stream);
+size_t lsh_local_bwd_workspace_size(const lsh_problem* p, int32_t n_back, int32_t n_fwd);
+lsh_status lsh_local_attn_bwd(const lsh_problem* p, int32_t n_back, int32_t n_fwd, const void* qk,
+                              const void* v, const void* out, const void* out_lo, const float* lse,
+                              const void* dout, float* dqk, float* dv, void* ws, size_t ws_bytes,
+                              lsh_stream_t stream);
+
+/*
  * lsh_sort_noalloc — lsh_sort without a caller workspace. The reference pages
  *   have no counterpart: this entry point exists for callers that cannot
  *   obtain device memory for a workspace, such as a host framework that owns
@@ -149,7 +188,7 @@ lsh_status lsh_attn_bwd(const lsh_problem* p, const void* qk, const void* v,
  *   process exits.
  *   - Same arguments, result and checks as lsh_sort. A problem whose
  *     lsh_sort_workspace_size() exceeds the scratch returns LSH_ERR_WORKSPACE
- *     and launches nothing. (16 MiB covers, e.g., 8 heads x 4 rounds x 65536
+ *     and launches nothing. (16 MiB covers, e.g., 8 heads x 4 rounds x 2^20
  *     positions with 1024 buckets, or 2 x 524288 positions with 8192.)
  *   - All calls on a device share the one scratch array and it keeps the last
  *     call's contents; the sort clears what must start at zero itself. Calls
@@ -163,8 +202,23 @@ lsh_status lsh_attn_bwd(const lsh_problem* p, const void* qk, const void* v,
 lsh_status lsh_sort_noalloc(const lsh_problem* p, const int32_t* bucket, int32_t* perm,
                             lsh_stream_t stream);
 
+/*
+ * lsh_check_wait_timeout — a health check of the failure detection; the
+ *   pages have no counterpart. Launches one small kernel in which a single
+ *   thread waits, through the same bounded-wait routine as the tensor-core
+ *   kernels' pipeline barriers, on a shared-memory barrier that nothing ever
+ *   completes. After `limit_ns` nanoseconds of GPU global time (1 .. 1e9) the
+ *   wait gives up, LSH_ERR_TIMEOUT is recorded in the device status word
+ *   (unless an earlier error is there) and the kernel returns, leaving the
+ *   context usable. Read the result with lsh_device_status(). Returns
+ *   LSH_ERR_INVALID_ARG for a limit outside that range, LSH_ERR_CUDA if the
+ *   launch fails.
+ */
+lsh_status lsh_check_wait_timeout(uint64_t limit_ns, lsh_stream_t stream);
+
 /* Synchronises `stream`, returns and clears the current device's status
- * word (LSH_OK, LSH_ERR_TIMEOUT or LSH_ERR_DEVICE_CHECK). */
+ * word: LSH_OK, or the FIRST error a kernel recorded since the last read
+ * (LSH_ERR_TIMEOUT, LSH_ERR_DEVICE_CHECK or LSH_ERR_RANGE). */
 lsh_status lsh_device_status(lsh_stream_t stream);
 
 /* Static, NUL-terminated description of a status code. */

@@ -34,8 +34,9 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings():
     _ensure_built()
-    for code in range(7):
+    for code in range(8):
         assert _lib.status_string(code)
+    assert "fp16" in _lib.status_string(7)
     assert _lib.status_string(0) == "ok"
 
 
@@ -109,7 +110,7 @@ def test_workspace_sizes_grow_with_problem():
     _ensure_built()
     L = _lib.lib()
     a = _p()
-    b = _p(L=8192)   # spans several sort tiles
+    b = _p(L=262144)   # spans several sort blocks per segment
     for f in (L.lsh_sort_workspace_size, L.lsh_fwd_workspace_size, L.lsh_bwd_workspace_size):
         assert 0 < f(ctypes.byref(a)) < f(ctypes.byref(b))
         assert f(ctypes.byref(a)) % 256 == 0
@@ -120,3 +121,27 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(_lib, "LIB_PATH", "/nonexistent/liblsh.so")
     with pytest.raises(_lib.LshLibraryMissing):
         _lib.lib()
+
+
+def test_wait_timeout_check_rejects_bad_limits_before_launch():
+    _ensure_built()
+    L = _lib.lib()
+    assert L.lsh_check_wait_timeout(0, None) == 1               # LSH_ERR_INVALID_ARG
+    assert L.lsh_check_wait_timeout(2_000_000_000, None) == 1
+
+
+def test_local_attention_rejects_bad_arguments_before_launch():
+    _ensure_built()
+    L = _lib.lib()
+    p = _p(n_rounds=1)
+    assert L.lsh_local_fwd_workspace_size(ctypes.byref(p), 1, 0) > 0
+    assert L.lsh_local_fwd_workspace_size(ctypes.byref(p), -1, 0) == 0
+    assert L.lsh_local_bwd_workspace_size(ctypes.byref(_p(n_rounds=2)), 1, 0) == 0
+    args = [FAKE] * 5 + [FAKE, 1 << 30, None]
+    assert L.lsh_local_attn_fwd(ctypes.byref(_p(n_rounds=2)), 1, 0, *args) == 1
+    assert L.lsh_local_attn_fwd(ctypes.byref(p), 0, -3, *args) == 1
+    assert L.lsh_local_attn_fwd(ctypes.byref(p), 1, 0, FAKE, FAKE, FAKE, None, FAKE, FAKE, 16,
+                                None) == 3                       # workspace too small
+    empty = _p(n_rounds=1, B=0)
+    assert L.lsh_local_attn_fwd(ctypes.byref(empty), 1, 1, None, None, None, None, None, None, 0,
+                                None) == 0
