@@ -5,24 +5,20 @@
 // before chunking. Sorting stably by bucket is sorting by the packed key
 // (round, bucket, position), because positions arrive in increasing order.
 //
-// Counting sort in four passes over tiles of positions:
-//   1. per tile, how many positions of each bucket it holds:
-//      counts[seg][bucket][tile]. For n_buckets <= 4096 (tiles of 2048) a
-//      warp walks 256 consecutive positions 32 at a time and counts with
-//      __match_any_sync into per-warp 16-bit counters; for larger bucket
-//      counts (tiles of 4096) the tile's packed keys (bucket << 12 | local
-//      index) are sorted in shared memory by a bitonic network and stored;
-//   2. row_scan: for every (seg, bucket), exclusive scan over tiles, plus the
-//      bucket total;
-//   3. bucket_scan: for every seg, exclusive scan of bucket totals;
-//   4. scatter: slot = base[seg][b] + counts[seg][b][tile] + rank of the
-//      position among the tile's positions of bucket b; perm[seg][slot] =
-//      position. The warp path recomputes the ranks in position order (step
-//      by step, lanes in order, warps in order through an exclusive prefix
-//      of the per-warp counts); the bitonic path takes them from the sorted
-//      packed keys, whose local index breaks ties.
-// Ranks follow position order inside a tile and tiles are placed in position
-// order, so the whole sort is stable.
+// Counting sort. Two paths:
+//  * n_buckets <= 8192 (every shape the workloads use): two kernels over
+//    blocks of 8K-32K consecutive positions, one CTA each (see the warp path
+//    below): per-warp counts with __match_any_sync, CTA totals per bucket,
+//    then a scatter kernel that forms the bucket bases itself and places
+//    every position at its slot;
+//  * larger bucket counts: per 4096-position tile the packed keys
+//    (bucket << 12 | local index) are sorted in shared memory by a bitonic
+//    network; row_scan / bucket_scan form the bases; scatter places them.
+// Ranks follow position order inside a warp (lanes in order, steps in order),
+// across the warps of a block (exclusive prefix of their counts) and across
+// blocks (counts of the blocks before), so the whole sort is stable.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -73,7 +69,7 @@ tile_sort_kernel(const int32_t* __restrict__ bucket, uint32_t* __restrict__ sort
     if (i < n) {
       uint32_t b = (uint32_t)src[i];
       if (b >= (uint32_t)n_buckets) {   // out-of-range id: flag it, keep memory safe
-        if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
+        record_status(status, (int)LSH_ERR_DEVICE_CHECK);
         b = (uint32_t)n_buckets - 1;
       }
       key = (b << 12) | (uint32_t)i;
@@ -182,81 +178,161 @@ scatter_kernel(const uint32_t* __restrict__ sorted, const int32_t* __restrict__ 
 }
 
 // ---- warp-counting path (n_buckets <= kWarpMaxBuckets) --------------------
-constexpr int kWarpMaxBuckets = 4096;
-constexpr int kWarpsPerTile = 8;
-constexpr int kWarpKeys = 256;                        // positions per warp
-constexpr int kWTile = kWarpsPerTile * kWarpKeys;     // 2048 positions per tile
-constexpr size_t kWarpSmem = (size_t)kWarpsPerTile * kWarpMaxBuckets * 2 + kWarpMaxBuckets * 4;
+// A segment is cut into Q blocks of P consecutive positions, one CTA each;
+// warp w of a CTA owns PW consecutive positions of its block and counts them
+// into its own 16-bit counters cnt[w][bucket] with __match_any_sync (one
+// leader lane per distinct bucket of a step updates the counter).
+//   sort_count_kernel:   counts[seg][q][bucket] = CTA totals (every bucket
+//                        written, so no clearing pass is needed);
+//   sort_scatter_kernel: bucket bases of the segment (exclusive scan of the
+//                        totals over buckets) plus the counts of the blocks
+//                        before q, the per-warp runs inside the block, then
+//                        every position goes to its slot in position order.
+constexpr int kWarpMaxBuckets = 8192;
+constexpr int kSortSmemBudget = 200 * 1024;
 
-// Counts of each bucket among this warp's 256 positions into cnt[b] (16-bit).
-__device__ __forceinline__ void warp_count(const int32_t* __restrict__ src, int n, int w, int lane,
-                                           uint16_t* cnt, int n_buckets, int* status) {
-  for (int st = 0; st < kWarpKeys / 32; ++st) {
-    const int i = w * kWarpKeys + st * 32 + lane;
+struct WarpGeo {
+  int W;        // warps per CTA
+  int PW;       // positions per warp (multiple of 32)
+  int P;        // positions per CTA = W * PW
+  int Q;        // CTAs per segment
+  size_t smem;  // dynamic shared memory of the scatter kernel (the larger)
+};
+
+WarpGeo warp_geo(const lsh_problem& p) {
+  WarpGeo g;
+  const int nb = p.n_buckets;
+  g.W = (int)std::min<int64_t>(32, (kSortSmemBudget - 8 * (int64_t)nb) / (2 * (int64_t)nb));
+  // a few blocks per segment (at most ~16) of 8K..32K positions
+  int64_t P = std::min<int64_t>(32768, std::max<int64_t>(8192, ((int64_t)p.L + 15) / 16));
+  g.PW = (int)((P + 32 * g.W - 1) / (32 * g.W)) * 32;
+  g.P = g.W * g.PW;
+  g.Q = (int)(((int64_t)p.L + g.P - 1) / g.P);
+  g.smem = (size_t)g.W * nb * 2 + (size_t)nb * 8 + 64 * 4;
+  return g;
+}
+
+// Counts the buckets of this warp's positions [i0, i0 + PW) of the segment
+// (those below L) into cnt[bucket].
+__device__ __forceinline__ void warp_count(const int32_t* __restrict__ seg_bucket, int64_t i0,
+                                           int PW, int L, int lane, uint16_t* cnt,
+                                           int n_buckets, int* status) {
+  for (int st = 0; st < PW; st += 32) {
+    const int64_t i = i0 + st + lane;
     uint32_t b = 0xffffffffu;
-    if (i < n) {
-      b = (uint32_t)src[i];
+    if (i < L) {
+      b = (uint32_t)__ldg(seg_bucket + i);
       if (b >= (uint32_t)n_buckets) {
-        if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
+        record_status(status, (int)LSH_ERR_DEVICE_CHECK);
         b = (uint32_t)n_buckets - 1;
       }
     }
     const uint32_t peers = __match_any_sync(0xffffffffu, b);
-    const int leader = __ffs(peers) - 1;
-    if (i < n && lane == leader) cnt[b] = (uint16_t)(cnt[b] + __popc(peers));
+    if (i < L && lane == __ffs(peers) - 1) cnt[b] = (uint16_t)(cnt[b] + __popc(peers));
     __syncwarp();
   }
 }
 
-__global__ void __launch_bounds__(kWarpsPerTile * 32)
-warp_count_kernel(const int32_t* __restrict__ bucket, int32_t* __restrict__ counts, int L,
-                  int n_buckets, int tiles, int* status) {
-  extern __shared__ uint8_t sm[];
-  uint16_t* hist = reinterpret_cast<uint16_t*>(sm);     // [warps][n_buckets]
-  const int tile = blockIdx.x % tiles;
-  const int64_t seg = blockIdx.x / tiles;
-  const int64_t p0 = (int64_t)tile * kWTile;
-  const int n = min(kWTile, (int)(L - p0));
+__device__ __forceinline__ void zero_counters(uint16_t* cnt, int n) {
+  uint32_t* c32 = reinterpret_cast<uint32_t*>(cnt);   // n is even
+  for (int i = threadIdx.x; i < n / 2; i += blockDim.x) c32[i] = 0u;
+}
+
+__global__ void __launch_bounds__(1024)
+sort_count_kernel(const int32_t* __restrict__ bucket, int32_t* __restrict__ counts, int L,
+                  int n_buckets, int PW, int P, int Q, int* status) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  uint16_t* cnt = reinterpret_cast<uint16_t*>(sm);      // [W][n_buckets]
+  const int W = blockDim.x >> 5;
+  const int q = blockIdx.x % Q;
+  const int64_t seg = blockIdx.x / Q;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < kWarpsPerTile * n_buckets; i += blockDim.x) hist[i] = 0;
+  zero_counters(cnt, W * n_buckets);
   __syncthreads();
-  warp_count(bucket + seg * L + p0, n, w, lane, hist + w * n_buckets, n_buckets, status);
+  warp_count(bucket + seg * L, (int64_t)q * P + (int64_t)w * PW, PW, L, lane,
+             cnt + w * n_buckets, n_buckets, status);
   __syncthreads();
-  int32_t* out = counts + seg * n_buckets * (int64_t)tiles + tile;
+  int32_t* out = counts + (seg * Q + q) * (int64_t)n_buckets;
   for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
     int tot = 0;
-#pragma unroll
-    for (int ww = 0; ww < kWarpsPerTile; ++ww) tot += hist[ww * n_buckets + b];
-    out[(int64_t)b * tiles] = tot;
+    for (int ww = 0; ww < W; ++ww) tot += cnt[ww * n_buckets + b];
+    out[b] = tot;
   }
 }
 
-__global__ void __launch_bounds__(kWarpsPerTile * 32)
-warp_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restrict__ counts,
-                    const int32_t* __restrict__ base, int32_t* __restrict__ perm, int L,
-                    int n_buckets, int tiles) {
-  extern __shared__ uint8_t sm[];
-  uint16_t* cnt = reinterpret_cast<uint16_t*>(sm);      // [warps][n_buckets]
-  int32_t* off = reinterpret_cast<int32_t*>(sm + (size_t)kWarpsPerTile * n_buckets * 2);
-  const int tile = blockIdx.x % tiles;
-  const int64_t seg = blockIdx.x / tiles;
-  const int64_t p0 = (int64_t)tile * kWTile;
-  const int n = min(kWTile, (int)(L - p0));
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int32_t* src = bucket + seg * L + p0;
-  for (int i = threadIdx.x; i < kWarpsPerTile * n_buckets; i += blockDim.x) cnt[i] = 0;
-  for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
-    const int64_t row = seg * n_buckets + b;
-    off[b] = base[row] + counts[row * tiles + tile];
+// Exclusive scan of v[0, n) in place by the whole block (n <= blockDim * 32
+// per thread run); `red` holds 64 ints of scratch.
+__device__ __forceinline__ void block_exclusive_scan(int32_t* v, int n, int* red) {
+  const int T = blockDim.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const int per = (n + T - 1) / T;
+  const int lo = min(n, t * per), hi = min(n, lo + per);
+  int sum = 0;
+  for (int i = lo; i < hi; ++i) sum += v[i];
+  int x = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) red[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    const int nw = (T + 31) >> 5;
+    const int a = lane < nw ? red[lane] : 0;
+    int y = a;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int z = __shfl_up_sync(0xffffffffu, y, o);
+      if (lane >= o) y += z;
+    }
+    red[32 + lane] = y - a;   // exclusive prefix of the warp sums
   }
   __syncthreads();
-  warp_count(src, n, w, lane, cnt + w * n_buckets, n_buckets, nullptr);
+  int run = red[32 + w] + x - sum;
+  for (int i = lo; i < hi; ++i) {
+    const int c = v[i];
+    v[i] = run;
+    run += c;
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(1024)
+sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restrict__ counts,
+                    int32_t* __restrict__ perm, int L, int n_buckets, int PW, int P, int Q) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int W = blockDim.x >> 5;
+  uint16_t* cnt = reinterpret_cast<uint16_t*>(sm);                                // [W][nb]
+  int32_t* base = reinterpret_cast<int32_t*>(sm + (size_t)W * n_buckets * 2);     // [nb]
+  int32_t* pre = base + n_buckets;                                                 // [nb]
+  int* red = pre + n_buckets;                                                      // [64]
+  const int q = blockIdx.x % Q;
+  const int64_t seg = blockIdx.x / Q;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  zero_counters(cnt, W * n_buckets);
+  // totals of the segment per bucket, and the counts of the blocks before q
+  const int32_t* cs = counts + seg * Q * (int64_t)n_buckets;
+  for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
+    int tot = 0, before = 0;
+    for (int qq = 0; qq < Q; ++qq) {
+      const int c = __ldg(cs + (int64_t)qq * n_buckets + b);
+      tot += c;
+      if (qq < q) before += c;
+    }
+    base[b] = tot;
+    pre[b] = before;
+  }
+  __syncthreads();
+  block_exclusive_scan(base, n_buckets, red);
+  for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) base[b] += pre[b];
+  const int32_t* sb = bucket + seg * L;
+  const int64_t i0 = (int64_t)q * P + (int64_t)w * PW;
+  warp_count(sb, i0, PW, L, lane, cnt + w * n_buckets, n_buckets, nullptr);
   __syncthreads();
   // exclusive prefix over warps: cnt[w][b] becomes the start of warp w's run
   for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
     int acc = 0;
-#pragma unroll
-    for (int ww = 0; ww < kWarpsPerTile; ++ww) {
+    for (int ww = 0; ww < W; ++ww) {
       const int c = cnt[ww * n_buckets + b];
       cnt[ww * n_buckets + b] = (uint16_t)acc;
       acc += c;
@@ -265,19 +341,18 @@ warp_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restric
   __syncthreads();
   uint16_t* mine = cnt + w * n_buckets;
   int32_t* out = perm + seg * L;
-  for (int st = 0; st < kWarpKeys / 32; ++st) {
-    const int i = w * kWarpKeys + st * 32 + lane;
+  for (int st = 0; st < PW; st += 32) {
+    const int64_t i = i0 + st + lane;
     uint32_t b = 0xffffffffu;
-    if (i < n) {
-      b = (uint32_t)src[i];
+    if (i < L) {
+      b = (uint32_t)__ldg(sb + i);
       if (b >= (uint32_t)n_buckets) b = (uint32_t)n_buckets - 1;
     }
     const uint32_t peers = __match_any_sync(0xffffffffu, b);
-    const int leader = __ffs(peers) - 1;
     const int rank = __popc(peers & ((1u << lane) - 1u));
-    if (i < n) out[off[b] + mine[b] + rank] = (int32_t)(p0 + i);
+    if (i < L) out[base[b] + mine[b] + rank] = (int32_t)i;
     __syncwarp();
-    if (i < n && lane == leader) mine[b] = (uint16_t)(mine[b] + __popc(peers));
+    if (i < L && lane == __ffs(peers) - 1) mine[b] = (uint16_t)(mine[b] + __popc(peers));
     __syncwarp();
   }
 }
@@ -288,8 +363,9 @@ bool warp_path(const lsh_problem& p) { return p.n_buckets <= kWarpMaxBuckets; }
 
 size_t sort_ws_bytes(const lsh_problem& p) {
   const int64_t S = (int64_t)p.B * p.H * p.n_rounds;
-  const int64_t tiles = warp_path(p) ? (p.L + kWTile - 1) / kWTile : (p.L + kTile - 1) / kTile;
-  size_t b = warp_path(p) ? 0 : align_up((size_t)S * p.L * 4, 256);
+  if (warp_path(p)) return align_up((size_t)S * warp_geo(p).Q * p.n_buckets * 4, 256);
+  const int64_t tiles = (p.L + kTile - 1) / kTile;
+  size_t b = align_up((size_t)S * p.L * 4, 256);
   b += align_up((size_t)S * p.n_buckets * tiles * 4, 256);
   b += align_up((size_t)S * p.n_buckets * 4, 256);
   return b;
@@ -297,11 +373,17 @@ size_t sort_ws_bytes(const lsh_problem& p) {
 
 SortWs sort_ws_carve(const lsh_problem& p, void* ws) {
   const int64_t S = (int64_t)p.B * p.H * p.n_rounds;
-  const int64_t tiles = warp_path(p) ? (p.L + kWTile - 1) / kWTile : (p.L + kTile - 1) / kTile;
-  char* c = (char*)ws;
   SortWs w;
-  w.sorted = warp_path(p) ? nullptr : (uint32_t*)c;
-  if (!warp_path(p)) c += align_up((size_t)S * p.L * 4, 256);
+  char* c = (char*)ws;
+  if (warp_path(p)) {
+    w.sorted = nullptr;
+    w.counts = (int32_t*)c;
+    w.base = nullptr;
+    return w;
+  }
+  const int64_t tiles = (p.L + kTile - 1) / kTile;
+  w.sorted = (uint32_t*)c;
+  c += align_up((size_t)S * p.L * 4, 256);
   w.counts = (int32_t*)c;
   c += align_up((size_t)S * p.n_buckets * tiles * 4, 256);
   w.base = (int32_t*)c;
@@ -313,21 +395,20 @@ cudaError_t launch_sort(const lsh_problem& p, const int32_t* bucket, int32_t* pe
   const int64_t S = (int64_t)p.B * p.H * p.n_rounds;
   const int64_t rows = S * p.n_buckets;
   if (warp_path(p)) {
-    const int tiles = (p.L + kWTile - 1) / kWTile;
-    const size_t sm = (size_t)kWarpsPerTile * p.n_buckets * 2 + (size_t)p.n_buckets * 4;
-    cudaError_t e = cudaFuncSetAttribute(warp_count_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWarpSmem);
+    const WarpGeo g = warp_geo(p);
+    const size_t sm_count_k = (size_t)g.W * p.n_buckets * 2;
+    cudaError_t e = cudaFuncSetAttribute(sort_count_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_count_k);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(warp_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kWarpSmem);
+    e = cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)g.smem);
     if (e != cudaSuccess) return e;
-    warp_count_kernel<<<(unsigned)(S * tiles), kWarpsPerTile * 32, sm, s>>>(bucket, ws.counts, p.L,
-                                                                            p.n_buckets, tiles, status);
-    row_scan_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(ws.counts, ws.base, rows, tiles);
-    bucket_scan_kernel<<<(unsigned)S, 1024, 0, s>>>(ws.base, p.n_buckets);
-    warp_scatter_kernel<<<(unsigned)(S * tiles), kWarpsPerTile * 32, sm, s>>>(
-        bucket, ws.counts, ws.base, perm, p.L, p.n_buckets, tiles);
-    note_launch(4);
+    const unsigned grid = (unsigned)(S * g.Q);
+    sort_count_kernel<<<grid, g.W * 32, sm_count_k, s>>>(bucket, ws.counts, p.L, p.n_buckets,
+                                                         g.PW, g.P, g.Q, status);
+    sort_scatter_kernel<<<grid, g.W * 32, g.smem, s>>>(bucket, ws.counts, perm, p.L, p.n_buckets,
+                                                       g.PW, g.P, g.Q);
+    note_launch(2);
     return cudaGetLastError();
   }
   const int tiles = (p.L + kTile - 1) / kTile;

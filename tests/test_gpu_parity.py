@@ -24,6 +24,11 @@ CASES = {
     "enwik8-small": W["enwik8-64k-bf16"].with_sizes(H=2, L=4160),
     "imagenet-small": W["imagenet64-12k-bf16"].with_sizes(B=2, H=2, L=1536),
     "halfmillion-small": W["halfmillion-bf16"].with_sizes(H=1, L=8256, backward=True),
+    # non-causal on the tensor cores (chunk 64): odd chunk counts (a last pair
+    # with one chunk), several work units per segment, backward on
+    "bf16-noncausal-m64": W["batch-bf16-8x8x4096"].with_sizes(B=1, H=3, L=1728, n_rounds=3,
+                                                               causal=False, backward=True),
+    "enwik8-noncausal-m64": W["enwik8-64k-bf16"].with_sizes(H=2, L=4160, causal=False),
     # non-causal, chunk 128, odd chunk count
     "bf16-noncausal-m128": W["batch-bf16-8x8x4096"].with_sizes(B=1, H=3, L=1664, chunk=128,
                                                                 causal=False, backward=True),
@@ -105,3 +110,63 @@ def test_autograd_wrapper_matches_oracle():
     # bf16 gradients: the tolerance includes one bf16 rounding of the result
     assert np.abs(qk.grad.float().cpu().numpy() - ref["dqk"]).max() <= 4e-2
     assert np.abs(v.grad.float().cpu().numpy() - ref["dv"]).max() <= 4e-2
+
+
+@pytest.mark.gpu
+def test_autograd_wrapper_tensor_core_path():
+    """The autograd wrapper on a chunk-64 bf16 problem (tensor-core kernels),
+    against the oracle run on the bucket ids the GPU hash produced (so that a
+    near-tie cannot change the permutation between the two)."""
+    import torch
+    from efficient_transformer_lsh_b200.attention import LSHAttention, lsh_attention
+    from oracle import lsh_oracle as orc
+    w = W["batch-bf16-8x8x4096"].with_sizes(B=1, H=2, L=1472, n_rounds=2, backward=True)
+    inp = generate(w)
+    dev = torch.device("cuda")
+    put = lambda a: torch.from_numpy(a).to(dev).to(torch.bfloat16)
+    qk = put(inp["qk"]).requires_grad_(True)
+    v = put(inp["v"]).requires_grad_(True)
+    R = put(inp["R"])
+    run = LSHAttention(w.B, w.H, w.L, w.n_buckets, w.n_rounds, w.chunk, w.causal, "bf16")
+    gpu_bucket = run.hash(qk.detach(), R).cpu().numpy()
+    out, lse = lsh_attention(qk, v, R, w.n_buckets, w.chunk, w.causal, w.scale)
+    dO = torch.from_numpy(inp["dO"]).to(dev)
+    (out.float() * dO).sum().backward()
+    f64 = {k: a.astype(np.float64) for k, a in inp.items()}
+    perm = orc.sort_positions(gpu_bucket)
+    O, LSE = orc.forward(f64["qk"], f64["v"], perm, w.chunk, w.causal, w.scale)
+    dqk, dv = orc.backward(f64["qk"], f64["v"], perm, w.chunk, w.causal, w.scale, O, LSE,
+                           f64["dO"])
+    assert np.abs(out.detach().float().cpu().numpy() - O).max() <= 2e-2
+    # bf16 gradients: the tolerance includes one bf16 rounding of the result
+    assert np.abs(qk.grad.float().cpu().numpy() - dqk).max() <= 4e-2
+    assert np.abs(v.grad.float().cpu().numpy() - dv).max() <= 4e-2
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("B,H,n_r,L,nb", [
+    (1, 1, 1, 64, 2),            # one block, one warp with work
+    (2, 3, 2, 1472, 24),         # ragged last warp
+    (1, 2, 1, 8256, 8192),       # largest bucket count of the counting path, two blocks
+    (1, 8, 4, 65536, 1024),      # eight blocks per segment
+    (1, 1, 1, 65600, 16384),     # beyond 8192 buckets: the bitonic tile path
+])
+def test_sort_paths_bit_exact(B, H, n_r, L, nb):
+    """Both sort paths against numpy's stable argsort, on uniform buckets
+    plus a heavy bucket (every seventh position), bit for bit."""
+    import torch
+    from efficient_transformer_lsh_b200 import _lib
+    rng = np.random.default_rng(nb + L)
+    bucket = rng.integers(0, nb, size=(B, H, n_r, L), dtype=np.int32)
+    bucket[..., ::7] = rng.integers(0, 3, size=bucket[..., ::7].shape)
+    p = _lib.make_problem(B, H, L, 64, nb, n_r, 64, True, 0.125, "bf16")
+    dev = torch.device("cuda")
+    bt = torch.from_numpy(bucket).to(dev)
+    perm = torch.full_like(bt, -1)
+    n = _lib.lsh_sort_workspace_size(p)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    _lib.lsh_sort(p, bt, perm, ws, n)
+    torch.cuda.synchronize()
+    assert _lib.lsh_device_status() == 0
+    ref = np.argsort(bucket.reshape(-1, L), axis=1, kind="stable").reshape(bucket.shape)
+    assert np.array_equal(perm.cpu().numpy(), ref)

@@ -21,8 +21,9 @@ def _problem(B, H, L, n_buckets, n_rounds):
 
 
 def test_too_large_problem_is_rejected_before_launch():
-    # 8 heads x 4 rounds x 2^20 positions needs ~140 MB of sort scratch
-    p = _problem(1, 8, 1 << 20, 1024, 4)
+    # 8 heads x 4 rounds x 2^20 positions with 8192 buckets needs 32 MiB of
+    # sort scratch (per-block bucket counts)
+    p = _problem(1, 8, 1 << 20, 8192, 4)
     assert _lib.lsh_sort_workspace_size(p) > _lib.SORT_NOALLOC_SCRATCH_BYTES
     FAKE = 1 << 20
     assert _lib.lib().lsh_sort_noalloc(ctypes.byref(p), FAKE, FAKE, None) == 3  # LSH_ERR_WORKSPACE
@@ -35,9 +36,10 @@ def test_sort_noalloc_matches_sort_two_calls():
     import torch
     dev = torch.device("cuda")
     rng = np.random.default_rng(7)
-    # two different problems back to back: the second reuses the scratch
-    # that still holds the first one's counters
-    shapes = [(1, 8, 65536, 1024, 4), (2, 3, 12288 + 64, 192, 5)]
+    # different problems back to back: each reuses the scratch that still
+    # holds the previous one's counters; the last has more than 8192 buckets,
+    # so it takes the other sort path, which must clear its counters itself
+    shapes = [(1, 8, 65536, 1024, 4), (2, 3, 12288 + 64, 192, 5), (1, 2, 65536, 16384, 1)]
     for B, H, L, nb, nr in shapes:
         p = _problem(B, H, L, nb, nr)
         assert _lib.lsh_sort_workspace_size(p) <= _lib.SORT_NOALLOC_SCRATCH_BYTES
