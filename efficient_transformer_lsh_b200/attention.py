@@ -79,6 +79,48 @@ class LSHAttention:
         return self.dqk, self.dv
 
 
+class LocalAttention:
+    """Local chunked self-attention for one fixed shape: the queries of chunk c
+    attend to chunks c - n_back .. c + n_fwd (identity order, shared qk with
+    the self-mask). Buffers: out/out_lo [B,H,L,d], lse [B,H,L], dqk/dv
+    [B,H,L,d] float32, and the two workspaces."""
+
+    def __init__(self, B, H, L, chunk, n_back, n_fwd, causal, dtype="bf16", d=64,
+                 scale: Optional[float] = None, device="cuda"):
+        self.dtype = dtype
+        self.tdtype = _TORCH_DTYPE[dtype]
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        self.n_back, self.n_fwd = int(n_back), int(n_fwd)
+        self.p = _lib.make_problem(B, H, L, d, 2, 1, chunk, causal, scale, dtype)
+        self.shape = (B, H, L, d)
+        dev = torch.device(device)
+        self.out = torch.empty(self.shape, dtype=self.tdtype, device=dev)
+        self.out_lo = torch.empty(self.shape, dtype=self.tdtype, device=dev) if dtype == "bf16" \
+            else None
+        self.lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+        self.dqk = torch.empty(self.shape, dtype=torch.float32, device=dev)
+        self.dv = torch.empty(self.shape, dtype=torch.float32, device=dev)
+        self.ws_fwd_bytes = _lib.lsh_local_fwd_workspace_size(self.p, self.n_back, self.n_fwd)
+        self.ws_bwd_bytes = _lib.lsh_local_bwd_workspace_size(self.p, self.n_back, self.n_fwd)
+        if min(self.ws_fwd_bytes, self.ws_bwd_bytes) == 0 and B * H * L > 0:
+            raise _lib.LshError(1, "workspace size query (problem rejected)")
+        u8 = dict(dtype=torch.uint8, device=dev)
+        self.ws_fwd = torch.empty(max(1, self.ws_fwd_bytes), **u8)
+        self.ws_bwd = torch.empty(max(1, self.ws_bwd_bytes), **u8)
+
+    def forward(self, qk, v, stream=None):
+        _lib.lsh_local_attn_fwd(self.p, self.n_back, self.n_fwd, qk, v, self.out, self.out_lo,
+                                self.lse, self.ws_fwd, self.ws_fwd_bytes, stream)
+        return self.out, self.lse
+
+    def backward(self, qk, v, dout, stream=None):
+        _lib.lsh_local_attn_bwd(self.p, self.n_back, self.n_fwd, qk, v, self.out, self.out_lo,
+                                self.lse, dout, self.dqk, self.dv, self.ws_bwd, self.ws_bwd_bytes,
+                                stream)
+        return self.dqk, self.dv
+
+
 class _LSHAttentionFn(torch.autograd.Function):
     @staticmethod
     def forward(ctx, qk, v, R, runner: LSHAttention):

@@ -24,12 +24,14 @@ constexpr int kQ = 64;    // query rows per block
 constexpr int kK = 64;    // keys per tile
 constexpr int kP = kD + 1;  // padded shared-memory row (floats)
 
-// Reads perm[i]; an id outside [0, L) is recorded in the status word and
-// replaced by 0 so that no gather leaves the tensor.
+// Reads perm[i] (the identity order when pr is null); an id outside [0, L) is
+// recorded in the status word and replaced by 0 so that no gather leaves the
+// tensor.
 __device__ __forceinline__ int checked_pos(const int32_t* pr, int i, int L, int* status) {
+  if (!pr) return i;
   int q = pr[i];
   if ((unsigned)q >= (unsigned)L) {
-    if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
+    record_status(status, (int)LSH_ERR_DEVICE_CHECK);
     q = 0;
   }
   return q;
@@ -46,11 +48,15 @@ __device__ __forceinline__ void load_rows(float (*dst)[kP], const T* __restrict_
 }
 
 // Per-round forward. Writes o_r (normalised) and lse_r in original order.
+// The queries of sorted chunk c see the key slots of chunks [c - n_back,
+// c + n_fwd] (clipped to the segment): n_back = 1, n_fwd = 0 is the LSH
+// window; a null perm is the identity order (local attention).
 template <typename T>
 __global__ void __launch_bounds__(256)
 fwd_round_kernel(const T* __restrict__ qk, const T* __restrict__ v, const int32_t* __restrict__ perm,
                  float* __restrict__ opart, float* __restrict__ lsepart, int L, int m,
-                 int n_rounds, int64_t N, int causal, float scale_log2, int* status) {
+                 int n_rounds, int64_t N, int causal, float scale_log2, int n_back, int n_fwd,
+                 int* status) {
   extern __shared__ float smem[];
   float(*Qs)[kP] = reinterpret_cast<float(*)[kP]>(smem);
   float(*Ks)[kP] = Qs + kQ;
@@ -65,11 +71,12 @@ fwd_round_kernel(const T* __restrict__ qk, const T* __restrict__ v, const int32_
   const int64_t seg = blockIdx.x / qblocks;
   const int r = (int)(seg % n_rounds);
   const int64_t bh = seg / n_rounds;
-  const int32_t* pr = perm + seg * L;
+  const int32_t* pr = perm ? perm + seg * L : nullptr;
   const T* X = qk + bh * L * kD;
   const T* Vb = v + bh * L * kD;
   const int t0 = qb * kQ, c = t0 / m;
-  const int k_lo = max(0, (c - 1) * m), k_hi = (c + 1) * m;
+  const int k_lo = (int)max((int64_t)0, (int64_t)(c - n_back) * m);
+  const int k_hi = (int)min((int64_t)L, (int64_t)(c + 1 + n_fwd) * m);
 
   if (tid < kQ) qpos[tid] = checked_pos(pr, t0 + tid, L, status);
   __syncthreads();
@@ -227,7 +234,7 @@ __global__ void __launch_bounds__(256)
 combine_f16_kernel(const __half* __restrict__ opart, const float* __restrict__ lsepart,
                    const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ out,
                    __nv_bfloat16* __restrict__ out_lo, float* __restrict__ lse, int64_t N,
-                   int n_rounds) {
+                   int n_rounds, int* status) {
   const int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
   const int c8 = (threadIdx.x & 7) * 8;
   if (tok >= N) return;
@@ -273,6 +280,12 @@ combine_f16_kernel(const __half* __restrict__ opart, const float* __restrict__ l
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = fmaf(wgt, f[i], acc[i]);
   }
+  // per-round outputs pass through fp16: a value outside its range (or a
+  // non-finite input) leaves a non-finite result, which is reported
+  bool fin = isfinite(LSE);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) fin = fin && isfinite(acc[i]);
+  if (!fin) record_status(status, (int)LSH_ERR_RANGE);
   const uint4 hi = pack8_bf16(acc);
   *o16 = hi;
   if (out_lo) {
@@ -324,7 +337,7 @@ bwd_round_kernel(const T* __restrict__ qk, const T* __restrict__ v, const T* __r
                  const int32_t* __restrict__ perm, const float* __restrict__ lse,
                  const float* __restrict__ D, float* __restrict__ dqk, float* __restrict__ dv,
                  int L, int m, int n_rounds, int causal, float scale, float scale_log2,
-                 int* status) {
+                 int n_back, int n_fwd, int* status) {
   extern __shared__ float smem[];
   float(*Qs)[kP] = reinterpret_cast<float(*)[kP]>(smem);
   float(*Gs)[kP] = Qs + kQ;
@@ -342,14 +355,15 @@ bwd_round_kernel(const T* __restrict__ qk, const T* __restrict__ v, const T* __r
   const int qb = blockIdx.x % qblocks;
   const int64_t seg = blockIdx.x / qblocks;
   const int64_t bh = seg / n_rounds;
-  const int32_t* pr = perm + seg * L;
+  const int32_t* pr = perm ? perm + seg * L : nullptr;
   const T* X = qk + bh * L * kD;
   const T* Vb = v + bh * L * kD;
   const T* Gb = dout + bh * L * kD;
   float* dX = dqk + bh * L * kD;
   float* dV = dv + bh * L * kD;
   const int t0 = qb * kQ, c = t0 / m;
-  const int k_lo = max(0, (c - 1) * m), k_hi = (c + 1) * m;
+  const int k_lo = (int)max((int64_t)0, (int64_t)(c - n_back) * m);
+  const int k_hi = (int)min((int64_t)L, (int64_t)(c + 1 + n_fwd) * m);
 
   if (tid < kQ) {
     int q = checked_pos(pr, t0 + tid, L, status);
@@ -465,16 +479,18 @@ constexpr size_t kBwdSmem = (size_t)(4 * kQ + 2 * kK) * kP * 4 + (kQ + kK) * 4 +
 
 template <typename T>
 cudaError_t fwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* perm, T* out,
-                  T* out_lo, float* lse, const FwdWs& ws, int* status, cudaStream_t s) {
+                  T* out_lo, float* lse, const FwdWs& ws, int* status, cudaStream_t s,
+                  int n_back = 1, int n_fwd = 0, bool allow_tc = true) {
   const int64_t N = (int64_t)p.B * p.H * p.L;
   const int64_t blocks = (int64_t)p.B * p.H * p.n_rounds * (p.L / kQ);
   const unsigned cblocks = (unsigned)((N * 16 + 255) / 256);
-  cudaError_t e = launch_attn_fwd_tc(p, qk, v, perm, ws.opart, ws.lsepart, status, s);
+  cudaError_t e = allow_tc ? launch_attn_fwd_tc(p, qk, v, perm, ws.opart, ws.lsepart, status, s)
+                           : cudaErrorNotSupported;
   if (e == cudaSuccess) {
     // the tensor-core forward handles bf16 problems only
     combine_f16_kernel<<<(unsigned)((N * 8 + 255) / 256), 256, 0, s>>>(
         (const __half*)ws.opart, ws.lsepart, (const __nv_bfloat16*)v, (__nv_bfloat16*)out,
-        (__nv_bfloat16*)out_lo, lse, N, p.n_rounds);
+        (__nv_bfloat16*)out_lo, lse, N, p.n_rounds, status);
     note_launch();
     return cudaGetLastError();
   }
@@ -484,7 +500,7 @@ cudaError_t fwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* 
   if (e != cudaSuccess) return e;
   fwd_round_kernel<T><<<(unsigned)blocks, 256, kFwdSmem, s>>>(
       qk, v, perm, ws.opart, ws.lsepart, p.L, p.chunk, p.n_rounds, N, p.causal,
-      p.scale * kLog2e, status);
+      p.scale * kLog2e, n_back, n_fwd, status);
   combine_kernel<T, float><<<cblocks, 256, 0, s>>>(ws.opart, ws.lsepart, v, out, out_lo, lse, N,
                                                    p.n_rounds);
   note_launch(2);
@@ -494,29 +510,100 @@ cudaError_t fwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* 
 template <typename T>
 cudaError_t bwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* perm, const T* out,
                   const T* out_lo, const float* lse, const T* dout, float* dqk, float* dv, float* D, int* status,
-                  cudaStream_t s) {
+                  cudaStream_t s, int n_back = 1, int n_fwd = 0, bool allow_tc = true) {
   const int64_t N = (int64_t)p.B * p.H * p.L;
   const int64_t blocks = (int64_t)p.B * p.H * p.n_rounds * (p.L / kQ);
   cudaError_t e = cudaFuncSetAttribute(bwd_round_kernel<T>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem);
   if (e != cudaSuccess) return e;
-  const bool tc = bwd_tc_ws_bytes(p) > 0;
-  bwd_prep_kernel<T><<<(unsigned)((N * 16 + 255) / 256), 256, 0, s>>>(out, out_lo, dout, lse, D, dqk, dv,
-                                                                        N, !tc);
-  note_launch();
-  if (tc) {
-    e = launch_attn_bwd_tc(p, qk, v, dout, perm, lse, D, dqk, dv,
+  if (allow_tc && bwd_tc_ws_bytes(p) > 0) {
+    e = launch_attn_bwd_tc(p, qk, v, dout, out, out_lo, perm, lse, D, dqk, dv,
                            (char*)D + align_up((size_t)N * 4, 256), status, s);
     return e == cudaSuccess ? cudaGetLastError() : e;
   }
+  bwd_prep_kernel<T><<<(unsigned)((N * 16 + 255) / 256), 256, 0, s>>>(out, out_lo, dout, lse, D, dqk, dv,
+                                                                        N, true);
+  note_launch();
   bwd_round_kernel<T><<<(unsigned)blocks, 256, kBwdSmem, s>>>(
       qk, v, dout, perm, lse, D, dqk, dv, p.L, p.chunk, p.n_rounds, p.causal, p.scale,
-      p.scale * kLog2e, status);
+      p.scale * kLog2e, n_back, n_fwd, status);
   note_launch();
   return cudaGetLastError();
 }
 
 }  // namespace
+
+// ---- local attention: the same kernels in the identity order ------------
+namespace {
+
+__global__ void iota_kernel(int32_t* __restrict__ perm, int L, int64_t total) {
+  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (k < total) perm[k] = (int32_t)(k % L);
+}
+
+// Look-back 1 and no look-ahead is the LSH window: bf16 problems with chunk
+// 64 take the tensor-core kernels with an identity permutation.
+bool local_tc(const lsh_problem& p, int n_back, int n_fwd) {
+  return p.dtype == LSH_BF16 && p.chunk == 64 && n_back == 1 && n_fwd == 0 && p.scale > 0.f;
+}
+
+int32_t* fill_identity(const lsh_problem& p, void* at, cudaStream_t s) {
+  const int64_t total = (int64_t)p.B * p.H * p.L;
+  int32_t* perm = (int32_t*)at;
+  iota_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(perm, p.L, total);
+  note_launch();
+  return perm;
+}
+
+}  // namespace
+
+size_t local_fwd_ws_bytes(const lsh_problem& p, int n_back, int n_fwd) {
+  const size_t N = (size_t)p.B * p.H * p.L;
+  return fwd_ws_bytes(p) + (local_tc(p, n_back, n_fwd) ? align_up(N * 4, 256) : 0);
+}
+
+cudaError_t launch_local_fwd(const lsh_problem& p, int n_back, int n_fwd, const void* qk,
+                             const void* v, void* out, void* out_lo, float* lse, void* ws,
+                             int* status, cudaStream_t s) {
+  const FwdWs w = fwd_ws_carve(p, ws);
+  if (local_tc(p, n_back, n_fwd)) {
+    const int32_t* perm = fill_identity(p, (char*)ws + fwd_ws_bytes(p), s);
+    return fwd_t(p, (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, perm, (__nv_bfloat16*)out,
+                 (__nv_bfloat16*)out_lo, lse, w, status, s);
+  }
+  if (p.dtype == LSH_BF16)
+    return fwd_t(p, (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, (const int32_t*)nullptr,
+                 (__nv_bfloat16*)out, (__nv_bfloat16*)out_lo, lse, w, status, s, n_back, n_fwd,
+                 false);
+  return fwd_t(p, (const float*)qk, (const float*)v, (const int32_t*)nullptr, (float*)out,
+               (float*)nullptr, lse, w, status, s, n_back, n_fwd, false);
+}
+
+size_t local_bwd_ws_bytes(const lsh_problem& p, int n_back, int n_fwd) {
+  const size_t N = (size_t)p.B * p.H * p.L;
+  if (local_tc(p, n_back, n_fwd)) return bwd_ws_bytes(p) + align_up(N * 4, 256);
+  return align_up(N * 4, 256);
+}
+
+cudaError_t launch_local_bwd(const lsh_problem& p, int n_back, int n_fwd, const void* qk,
+                             const void* v, const void* out, const void* out_lo, const float* lse,
+                             const void* dout, float* dqk, float* dv, void* ws, int* status,
+                             cudaStream_t s) {
+  float* D = (float*)ws;
+  if (local_tc(p, n_back, n_fwd)) {
+    const int32_t* perm = fill_identity(p, (char*)ws + bwd_ws_bytes(p), s);
+    return bwd_t(p, (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, perm,
+                 (const __nv_bfloat16*)out, (const __nv_bfloat16*)out_lo, lse,
+                 (const __nv_bfloat16*)dout, dqk, dv, D, status, s);
+  }
+  if (p.dtype == LSH_BF16)
+    return bwd_t(p, (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, (const int32_t*)nullptr,
+                 (const __nv_bfloat16*)out, (const __nv_bfloat16*)out_lo, lse,
+                 (const __nv_bfloat16*)dout, dqk, dv, D, status, s, n_back, n_fwd, false);
+  return bwd_t(p, (const float*)qk, (const float*)v, (const int32_t*)nullptr, (const float*)out,
+               (const float*)nullptr, lse, (const float*)dout, dqk, dv, D, status, s, n_back, n_fwd,
+               false);
+}
 
 size_t fwd_ws_bytes(const lsh_problem& p) {
   const size_t N = (size_t)p.B * p.H * p.L;

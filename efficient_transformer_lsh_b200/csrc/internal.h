@@ -54,22 +54,34 @@ cudaError_t launch_attn_fwd_tc(const lsh_problem& p, const void* qk, const void*
                                const int32_t* perm, void* opart_f16, float* lsepart, int* status,
                                cudaStream_t s);
 
-// tcgen05 backward (bf16, chunk 64): writes dqk and dv (every element, the
-// self-attending rows' dout included) from D = dout . out; `ws` holds
-// bwd_tc_ws_bytes(p) bytes (inverse permutation, per-round fp16 partials).
+// tcgen05 backward (bf16, chunk 64): forms D = dout . (out + out_lo) into D
+// and fp16 copies of qk, v, dout, then writes dqk and dv (every element, the
+// self-attending rows' dout included); `ws` holds bwd_tc_ws_bytes(p) bytes
+// (fp16 copies, inverse permutation, per-round fp16 partials).
 // bwd_tc_ws_bytes is 0 and the launcher returns cudaErrorNotSupported for
 // other problems.
 size_t bwd_tc_ws_bytes(const lsh_problem& p);
 cudaError_t launch_attn_bwd_tc(const lsh_problem& p, const void* qk, const void* v,
-                               const void* dout, const int32_t* perm, const float* lse,
-                               const float* D, float* dqk, float* dv, void* ws, int* status,
-                               cudaStream_t s);
+                               const void* dout, const void* out, const void* out_lo,
+                               const int32_t* perm, const float* lse, float* D, float* dqk,
+                               float* dv, void* ws, int* status, cudaStream_t s);
 
 size_t bwd_ws_bytes(const lsh_problem& p);
 cudaError_t launch_attn_bwd(const lsh_problem& p, const void* qk, const void* v,
                             const int32_t* perm, const void* out, const void* out_lo,
                             const float* lse, const void* dout, float* dqk, float* dv, void* ws,
                             int* status, cudaStream_t s);
+
+// ---- local attention (identity order, n_back / n_fwd chunks of overlap) ----
+size_t local_fwd_ws_bytes(const lsh_problem& p, int n_back, int n_fwd);
+cudaError_t launch_local_fwd(const lsh_problem& p, int n_back, int n_fwd, const void* qk,
+                             const void* v, void* out, void* out_lo, float* lse, void* ws,
+                             int* status, cudaStream_t s);
+size_t local_bwd_ws_bytes(const lsh_problem& p, int n_back, int n_fwd);
+cudaError_t launch_local_bwd(const lsh_problem& p, int n_back, int n_fwd, const void* qk,
+                             const void* v, const void* out, const void* out_lo, const float* lse,
+                             const void* dout, float* dqk, float* dv, void* ws, int* status,
+                             cudaStream_t s);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
