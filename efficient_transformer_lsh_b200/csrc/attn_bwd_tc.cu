@@ -39,14 +39,15 @@
 // item all run at once.
 //
 // Warp roles (persistent CTA, one per SM), register budgets via setmaxnreg:
-//   warps 0-2  : producers — cp.async gathers of x, dout (3 chunks) and v
-//                (2 chunks) into a 2-slot ring, in-place bf16 -> fp16
-//                conversion, per-query position, log2-scaled LSE and D;
+//   warps 0-2  : producers — cp.async gathers of the fp16 copies of x, dout
+//                (3 chunks) and v (2 chunks) into a 2-slot ring, per-query
+//                position, log2-scaled LSE and D;
 //   warp 3     : TMEM allocation and the MMA-issuing thread;
 //   warps 4-7  : gradient flush of the previous item (one thread per row,
 //                fp16 staging in shared memory, TMA stores);
-//   warps 8-11, 12-15: two softmax warpgroups, one per S^T buffer (even and
-//                odd steps), one thread per key row.
+//   warps 8-23 : four softmax warpgroups, two per S^T buffer (even and odd
+//                steps), one thread per key row and 32 of the block's 64
+//                query columns each.
 #include <cuda_fp16.h>
 #include <stddef.h>
 
@@ -70,10 +71,14 @@ constexpr int kSlotBytes = 8 * kTile;  // 64 KB
 constexpr int kDsBlock = 128 * 128;    // 128 key rows x 64 query columns
 constexpr int kDsBytes = 4 * kDsBlock; // dS^T blocks 0,1,2 + a zero block
 constexpr int kStageBytes = 128 * 128; // 128 fp16 rows, 128-byte swizzle
-constexpr int kThreads = 512;
+constexpr int kThreads = 768;
 constexpr int kProducers = 96;
-constexpr int kRegsLow = 104, kRegsFlush = 88, kRegsSmx = 144;
-static_assert(128 * (kRegsLow + kRegsFlush) + 256 * kRegsSmx <= kThreads * 128, "register split");
+// Launched at 80 registers per thread (768 threads); producers/MMA and flush
+// drop to 48, the four softmax warpgroups rise to 96.
+constexpr int kRegsLaunch = 80;
+constexpr int kRegsLow = 48, kRegsFlush = 48, kRegsSmx = 96;
+static_assert(128 * (kRegsLow + kRegsFlush) + 512 * kRegsSmx <= kThreads * kRegsLaunch,
+              "register split");
 // TMEM columns
 constexpr uint32_t kColBuf = 0;        // + 128 w: S^T (64) | dP^T (64); P^T over S^T
 constexpr uint32_t kColAcc = 256;      // + 128 a: dV (64) | dK (64)
@@ -146,56 +151,21 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 // one lane never leaves the others inside a warp-collective instruction.
 __device__ __forceinline__ bool warp_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
 
-__device__ __forceinline__ void issue_row(const __nv_bfloat16* __restrict__ src_row, uint8_t* tile,
-                                          int row, int half) {
-  const uint32_t base = smem_u32(tile) + row * 128;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int ch = half * 4 + i;
-    cp_async16(base + (((uint32_t)ch ^ (uint32_t)(row & 7)) << 4), src_row + ch * 8);
-  }
-}
-__device__ __forceinline__ void convert_row(uint8_t* tile, int row, int half) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int ch = half * 4 + i;
-    convert_piece_bf16_to_f16(tile + row * 128 + ((ch ^ (row & 7)) << 4));
-  }
-}
-
-// A wait's outcome made uniform across the `n` threads of named barrier `id`
-// (all of them must call it).
-__device__ __forceinline__ bool group_ok(int id, int n, bool ok) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "barrier.red.and.pred po, %2, %3, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)ok), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
-__device__ __forceinline__ void named_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
 // Converts 64 fp32 TMEM columns of this thread's lane, times `sc`, to fp16
 // and writes them as row `row` of a 128-byte-swizzled staging tile.
 __device__ __forceinline__ void stage_row(uint32_t ta, float sc, uint8_t* stage, int row) {
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t a[32];
-    tmem_ld32(ta + 32 * h, a);
+  for (int h = 0; h < 4; ++h) {
+    uint32_t a[16];
+    tmem_ld16(ta + 16 * h, a);
     tmem_ld_wait();
-    uint32_t pk[16];
+    uint32_t pk[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < 8; ++i)
       pk[i] = pack_f16x2(__uint_as_float(a[2 * i]) * sc, __uint_as_float(a[2 * i + 1]) * sc);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int ch = h * 4 + c;
+    for (int c = 0; c < 2; ++c) {
+      const int ch = h * 2 + c;
       *reinterpret_cast<uint4*>(stage + row * 128 + ((ch ^ (row & 7)) << 4)) =
           make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
     }
@@ -229,20 +199,22 @@ __device__ __forceinline__ void bwd_issue_g(uint32_t tmem, uint32_t acc, uint32_
                                             bool acc_v, bool acc_k) {
   const uint32_t pt = tmem + kColBuf + (uint32_t)(g & 1) * 128;
   const uint32_t gq = sl + (kDo + qb * kTile) / 16 + kLboN, xq = sl + (kX + qb * kTile) / 16 + kLboN;
+  // packed queries 0-31 sit at columns 0-15, queries 32-63 at columns 32-47
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks) {
-    mma_ts_w(acc, pt + ks * 8, gq + 128 * ks, kDescHi1024, kIdKN, acc_v || ks > 0);
-    mma_ts_w(acc + 64, pt + 64 + ks * 8, xq + 128 * ks, kDescHi1024, kIdKN, acc_k || ks > 0);
+    const uint32_t ca = 8 * ks + 16 * (ks >> 1);
+    mma_ts_w(acc, pt + ca, gq + 128 * ks, kDescHi1024, kIdKN, acc_v || ks > 0);
+    mma_ts_w(acc + 64, pt + 64 + ca, xq + 128 * ks, kDescHi1024, kIdKN, acc_k || ks > 0);
   }
 }
 // Query-side product dS[128 queries of the dS^T blocks at ds] X_K over the
-// first 16 KS keys, into the dK columns at d.
-template <int KS>
+// keys [16 KS0, 16 KS1), into the dK columns at d.
+template <int KS0, int KS1>
 __device__ __forceinline__ void bwd_issue_r(uint32_t d, uint32_t ds, uint32_t sl, bool acc) {
   const uint32_t xk = sl + kX / 16 + kLboN;
 #pragma unroll
-  for (int ks = 0; ks < KS; ++ks)
-    mma_ss_w(d, ds + 128 * ks, xk + 128 * ks, kDescHi1024, kIdNN, acc || ks > 0);
+  for (int ks = KS0; ks < KS1; ++ks)
+    mma_ss_w(d, ds + 128 * ks, xk + 128 * ks, kDescHi1024, kIdNN, acc || ks > KS0);
 }
 __device__ __forceinline__ bool bwd_wait_p(BwdBar* bar, int g, volatile int* abort, int* status) {
   return mbar_wait(&bar->p_full[g & 1], (uint32_t)(g >> 1) & 1u, abort, status);
@@ -250,8 +222,8 @@ __device__ __forceinline__ bool bwd_wait_p(BwdBar* bar, int g, volatile int* abo
 
 template <bool kCausal>
 __global__ void __launch_bounds__(kThreads, 1)
-attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __restrict__ v,
-                   const __nv_bfloat16* __restrict__ dout, const int32_t* __restrict__ perm,
+attn_bwd_tc_kernel(const __half* __restrict__ qk, const __half* __restrict__ v,
+                   const __half* __restrict__ dout, const int32_t* __restrict__ perm,
                    const float* __restrict__ lse, const float* __restrict__ Dg,
                    const __grid_constant__ CUtensorMap map_dv,
                    const __grid_constant__ CUtensorMap map_dqk,
@@ -277,7 +249,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bar->s_full[w], 1);
-      mbar_init(&bar->p_full[w], 128);
+      mbar_init(&bar->p_full[w], 256);
       mbar_init(&bar->g_full[w], 1);
       mbar_init(&bar->acc_free[w], 128);
     }
@@ -334,14 +306,14 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
         const bool live = c < min(3, n_chunks - 2 * j.p);
         uint8_t* sl = slots + s * kSlotBytes;
         if ((unsigned)pa >= (unsigned)L || (unsigned)pb >= (unsigned)L) {
-          if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
+          record_status(status, (int)LSH_ERR_DEVICE_CHECK);
           if ((unsigned)pa >= (unsigned)L) pa = 0;
           if ((unsigned)pb >= (unsigned)L) pb = 0;
         }
         if (live) {
-          const __nv_bfloat16* xb = qk + bh * L * 64 + ch * 8;
-          const __nv_bfloat16* gb = dout + bh * L * 64 + ch * 8;
-          const __nv_bfloat16* vb = v + bh * L * 64 + ch * 8;
+          const __half* xb = qk + bh * L * 64 + ch * 8;
+          const __half* gb = dout + bh * L * 64 + ch * 8;
+          const __half* vb = v + bh * L * 64 + ch * 8;
           const uint32_t tx = smem_u32(sl + kX + c * kTile), tg = smem_u32(sl + kDo + c * kTile),
                          tv = smem_u32(sl + kV + c * kTile);
 #pragma unroll
@@ -374,16 +346,6 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
           bar->tok[n & 3][q] = tp;
         }
         cp_async_wait<0>();
-        if (live) {
-#pragma unroll
-          for (int g = 0; g < 16; ++g) {
-            const int row = 4 * g + rsub;
-            const uint32_t off = row * 128 + (((uint32_t)ch ^ (uint32_t)(row & 7)) << 4);
-            convert_piece_bf16_to_f16(sl + kX + c * kTile + off);
-            convert_piece_bf16_to_f16(sl + kDo + c * kTile + off);
-            if (c < 2) convert_piece_bf16_to_f16(sl + kV + c * kTile + off);
-          }
-        }
         fence_proxy_async();
         mbar_arrive(&bar->slot_full[s]);
         j = jn;
@@ -442,8 +404,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
         if (!bwd_wait_p(bar, g0 + 1, abort, status)) break;
         tc_fence_after();
         bwd_issue_g(tmem, acc, sl, g0 + 1, 0, nc > 1, nc > 1 || !cur.first);
-        if (nc >= 2) bwd_issue_r<8>(acc + 64, ds_lo, sl, true);
-        else bwd_issue_r<4>(acc + 64, ds_lo, sl, true);
+        if (nc >= 2) bwd_issue_r<0, 8>(acc + 64, ds_lo, sl, true);
+        else bwd_issue_r<0, 4>(acc + 64, ds_lo, sl, true);
         int nc_next = 0;
         uint32_t sl_next = 0;
         if (have_next) {
@@ -466,8 +428,10 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
             ok = mbar_wait(&bar->acc_free[b], (uint32_t)(seen_b++) & 1u, abort, status);
           if (!ok) break;
           tc_fence_after();
-          bwd_issue_r<8>(tmem + kColAcc + (uint32_t)b * 128 + 64, ds_lo + 2 * (kDsBlock / 16), sl,
-                         false);
+          // block 2's queries see only the keys of chunk 2p+1 (rows 64-127;
+          // the other rows of the block hold zeros)
+          bwd_issue_r<4, 8>(tmem + kColAcc + (uint32_t)b * 128 + 64, ds_lo + 2 * (kDsBlock / 16), sl,
+                            false);
         }
         mma_commit(&bar->g_full[a]);
         mma_commit(&bar->slot_free[s]);
@@ -534,11 +498,17 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
     if (issuer) bulk_wait_all();
   } else {
     // ------------------------------------------------ softmax: P^T and dS^T
+    // Two warpgroups per S^T buffer, each owning 32 of the block's 64 query
+    // columns; each writes its packed P^T / dS^T inside its own half of the
+    // buffer's columns, so neither overwrites columns the other still reads.
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSmx));
-    const int w = wgi - 2;                     // S^T buffer = parity of the step
+    const int sw = wgi - 2;
+    const int w = sw >> 1;                     // S^T buffer = parity of the step
+    const int hc = sw & 1;                     // column half of the block
     const int q = warp & 3;
     const int row = q * 32 + lane;             // key row = TMEM lane
-    const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + kColBuf + (uint32_t)w * 128;
+    const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + kColBuf + (uint32_t)w * 128 +
+                        (uint32_t)(32 * hc);
     JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
     Job j;
     int n = 0, k = 0;
@@ -566,14 +536,14 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
             const float* d_all = bar->dval[s];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int col0 = qb * 64 + h * 32;
-              uint32_t sv[32], pv[32];
-              tmem_ld32(tb + h * 32, sv);
-              tmem_ld32(tb + 64 + h * 32, pv);
+              const int col0 = qb * 64 + 32 * hc + 16 * h;
+              uint32_t sv[16], pv[16];
+              tmem_ld16(tb + 16 * h, sv);
+              tmem_ld16(tb + 64 + 16 * h, pv);
               tmem_ld_wait();
-              uint32_t pk[16], dk[16];
+              uint32_t pk[8], dk[8];
 #pragma unroll
-              for (int i4 = 0; i4 < 8; ++i4) {
+              for (int i4 = 0; i4 < 4; ++i4) {
                 const int4 q4 = *reinterpret_cast<const int4*>(qp_all + col0 + 4 * i4);
                 const float4 l4 = *reinterpret_cast<const float4*>(l2_all + col0 + 4 * i4);
                 const float4 d4 = *reinterpret_cast<const float4*>(d_all + col0 + 4 * i4);
@@ -595,27 +565,28 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
                 dk[2 * i4] = pack_f16x2(de[0], de[1]);
                 dk[2 * i4 + 1] = pack_f16x2(de[2], de[3]);
               }
-              // P^T and dS^T over the S^T / dP^T columns already read; dS^T
-              // also into shared memory
-              tmem_st16(tb + h * 16, pk);
-              tmem_st16(tb + 64 + h * 16, dk);
+              // packed P^T and dS^T over this half's S^T / dP^T columns that
+              // are already read; dS^T also into shared memory
+              tmem_st8(tb + 8 * h, pk);
+              tmem_st8(tb + 64 + 8 * h, dk);
 #pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const int ch = h * 4 + c;
+              for (int c = 0; c < 2; ++c) {
+                const int ch = 4 * hc + 2 * h + c;
                 *reinterpret_cast<uint4*>(drow + ((ch ^ (row & 7)) << 4)) =
                     make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
               }
             }
           } else {
             // a key row that this query block does not see: P = 0 and dS = 0
-            uint32_t z[32];
+            uint32_t z[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) z[e] = 0u;
-            tmem_st32(tb, z);
-            tmem_st32(tb + 64, z);
+            for (int e = 0; e < 16; ++e) z[e] = 0u;
+            tmem_st16(tb, z);
+            tmem_st16(tb + 64, z);
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-              *reinterpret_cast<uint4*>(drow + ((ch ^ (row & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+            for (int c = 0; c < 4; ++c)
+              *reinterpret_cast<uint4*>(drow + (((4 * hc + c) ^ (row & 7)) << 4)) =
+                  make_uint4(0u, 0u, 0u, 0u);
           }
           tmem_st_wait();
           fence_proxy_async();
@@ -634,6 +605,51 @@ attn_bwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
   }
 }
 
+// D_i = dout_i . (out_i + out_lo_i), and fp16 copies of qk, v and dout for the
+// tensor-core products (exact for values inside the fp16 range; a value
+// outside it becomes inf, which the check of the results reports). Eight
+// threads per token, 16 bytes of each tensor per thread.
+__global__ void __launch_bounds__(256)
+bwd_prep_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __restrict__ v,
+                   const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out,
+                   const __nv_bfloat16* __restrict__ out_lo, float* __restrict__ D,
+                   __half* __restrict__ x16, __half* __restrict__ v16, __half* __restrict__ g16,
+                   int64_t N) {
+  const int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
+  const int c8 = (threadIdx.x & 7) * 8;
+  const bool live = tok < N;
+  const int64_t off = (live ? tok : 0) * 64 + c8;
+  uint4 o = make_uint4(0u, 0u, 0u, 0u), lo = o, g = o, x = o, w = o;
+  if (live) {
+    o = __ldg(reinterpret_cast<const uint4*>(out + off));
+    if (out_lo) lo = __ldg(reinterpret_cast<const uint4*>(out_lo + off));
+    g = __ldg(reinterpret_cast<const uint4*>(dout + off));
+    x = __ldg(reinterpret_cast<const uint4*>(qk + off));
+    w = __ldg(reinterpret_cast<const uint4*>(v + off));
+  }
+  const uint32_t ou[4] = {o.x, o.y, o.z, o.w}, lu[4] = {lo.x, lo.y, lo.z, lo.w};
+  const uint32_t gu[4] = {g.x, g.y, g.z, g.w};
+  float d = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float o0 = __uint_as_float(ou[i] << 16) + __uint_as_float(lu[i] << 16);
+    const float o1 = __uint_as_float(ou[i] & 0xffff0000u) + __uint_as_float(lu[i] & 0xffff0000u);
+    d = fmaf(o0, __uint_as_float(gu[i] << 16), d);
+    d = fmaf(o1, __uint_as_float(gu[i] & 0xffff0000u), d);
+  }
+  d += __shfl_xor_sync(0xffffffffu, d, 4);
+  d += __shfl_xor_sync(0xffffffffu, d, 2);
+  d += __shfl_xor_sync(0xffffffffu, d, 1);
+  if (!live) return;
+  if (c8 == 0) D[tok] = d;
+  *reinterpret_cast<uint4*>(x16 + off) = make_uint4(bf16x2_to_f16x2(x.x), bf16x2_to_f16x2(x.y),
+                                                    bf16x2_to_f16x2(x.z), bf16x2_to_f16x2(x.w));
+  *reinterpret_cast<uint4*>(v16 + off) = make_uint4(bf16x2_to_f16x2(w.x), bf16x2_to_f16x2(w.y),
+                                                    bf16x2_to_f16x2(w.z), bf16x2_to_f16x2(w.w));
+  *reinterpret_cast<uint4*>(g16 + off) = make_uint4(bf16x2_to_f16x2(g.x), bf16x2_to_f16x2(g.y),
+                                                    bf16x2_to_f16x2(g.z), bf16x2_to_f16x2(g.w));
+}
+
 // inv[seg][perm[seg][i]] = i: the slot of every position in every round.
 __global__ void __launch_bounds__(256)
 inverse_perm_kernel(const int32_t* __restrict__ perm, int32_t* __restrict__ inv, int L,
@@ -644,14 +660,13 @@ inverse_perm_kernel(const int32_t* __restrict__ perm, int32_t* __restrict__ inv,
   const int i = (int)(k - seg * L);
   const int pos = perm[k];
   if ((unsigned)pos >= (unsigned)L) {
-    if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
+    record_status(status, (int)LSH_ERR_DEVICE_CHECK);
     return;
   }
   inv[seg * L + pos] = i;
 }
 
-__device__ __forceinline__ void add8_f16(float (&acc)[8], const __half* src) {
-  const uint4 w = *reinterpret_cast<const uint4*>(src);
+__device__ __forceinline__ void add8_f16(float (&acc)[8], const uint4 w) {
   const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -664,7 +679,9 @@ __device__ __forceinline__ void add8_f16(float (&acc)[8], const __half* src) {
 // dv, dqk of every token: the sum over rounds of its partial rows (slot
 // inv[seg][pos] of segment seg = bh * n_rounds + r), plus the unit-end R1
 // row where its slot opens a unit; dv also takes dout for a token that
-// attended only to itself (final LSE of -inf). Eight threads per token.
+// attended only to itself (final LSE of -inf). Eight threads per token;
+// the slots of two rounds are looked up first and their four rows loaded
+// together, to keep more reads in flight.
 __global__ void __launch_bounds__(256)
 unsort_kernel(const __half* __restrict__ part_dv, const __half* __restrict__ part_dqk,
               const __half* __restrict__ edge, const int32_t* __restrict__ inv,
@@ -679,20 +696,32 @@ unsort_kernel(const __half* __restrict__ part_dv, const __half* __restrict__ par
   float a[8], b[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) a[e] = b[e] = 0.f;
-  for (int r = 0; r < n_rounds; ++r) {
-    const int64_t seg = bh * n_rounds + r;
-    const int i = inv[seg * L + pos];
-    if ((unsigned)i >= (unsigned)L) {
-      if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
-      continue;
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  for (int r0 = 0; r0 < n_rounds; r0 += 2) {
+    int slot[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+      slot[k] = r0 + k < n_rounds ? __ldg(inv + (bh * n_rounds + r0 + k) * L + pos) : 0;
+    uint4 ua[2], ub[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const bool live = r0 + k < n_rounds;
+      const bool ok = (unsigned)slot[k] < (unsigned)L;
+      if (live && !ok) record_status(status, (int)LSH_ERR_DEVICE_CHECK);
+      const int64_t row = (bh * n_rounds + r0 + k) * L + (ok ? slot[k] : 0);
+      ua[k] = live && ok ? __ldg(reinterpret_cast<const uint4*>(part_dv + row * 64 + c8)) : zero;
+      ub[k] = live && ok ? __ldg(reinterpret_cast<const uint4*>(part_dqk + row * 64 + c8)) : zero;
     }
-    const int64_t row = seg * L + i;
-    add8_f16(a, part_dv + row * 64 + c8);
-    add8_f16(b, part_dqk + row * 64 + c8);
-    const int c = i / kM;
-    if (c > 0 && c % (2 * kUnit) == 0) {
-      const int64_t er = (seg * units_per_seg + c / (2 * kUnit) - 1) * kM + (i % kM);
-      add8_f16(b, edge + er * 64 + c8);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      add8_f16(a, ua[k]);
+      add8_f16(b, ub[k]);
+      const int i = slot[k], c = i / kM;
+      if (r0 + k < n_rounds && (unsigned)i < (unsigned)L && c > 0 && c % (2 * kUnit) == 0) {
+        const int64_t er = ((bh * n_rounds + r0 + k) * units_per_seg + c / (2 * kUnit) - 1) * kM +
+                           (i % kM);
+        add8_f16(b, __ldg(reinterpret_cast<const uint4*>(edge + er * 64 + c8)));
+      }
     }
   }
   if (lse[t] == -INFINITY) {
@@ -704,6 +733,12 @@ unsort_kernel(const __half* __restrict__ part_dv, const __half* __restrict__ par
       a[2 * i + 1] += __uint_as_float(u[i] & 0xffff0000u);
     }
   }
+  // the partial rows are fp16: a value outside its range (or a non-finite
+  // input) leaves a non-finite gradient, which is reported
+  bool fin = true;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) fin = fin && isfinite(a[e]) && isfinite(b[e]);
+  if (!fin) record_status(status, (int)LSH_ERR_RANGE);
   float4* pv = reinterpret_cast<float4*>(dv + t * 64 + c8);
   float4* pq = reinterpret_cast<float4*>(dqk + t * 64 + c8);
   pv[0] = make_float4(a[0], a[1], a[2], a[3]);
@@ -721,6 +756,9 @@ bool tc_eligible(const lsh_problem& p) {
 }
 
 struct TcWs {
+  __half* x16;
+  __half* v16;
+  __half* g16;
   int32_t* inv;
   __half* part_dv;
   __half* part_dqk;
@@ -736,6 +774,13 @@ TcWs tc_ws(const lsh_problem& p, void* base) {
   TcWs w;
   char* c = (char*)base;
   size_t off = 0;
+  const size_t toks = (size_t)p.B * p.H * p.L;
+  w.x16 = (__half*)(c + off);
+  off += al(toks * 64 * 2);
+  w.v16 = (__half*)(c + off);
+  off += al(toks * 64 * 2);
+  w.g16 = (__half*)(c + off);
+  off += al(toks * 64 * 2);
   w.inv = (int32_t*)(c + off);
   off += al(rows * 4);
   w.part_dv = (__half*)(c + off);
@@ -755,9 +800,9 @@ size_t bwd_tc_ws_bytes(const lsh_problem& p) {
 }
 
 cudaError_t launch_attn_bwd_tc(const lsh_problem& p, const void* qk, const void* v,
-                               const void* dout, const int32_t* perm, const float* lse,
-                               const float* D, float* dqk, float* dv, void* ws, int* status,
-                               cudaStream_t s) {
+                               const void* dout, const void* out, const void* out_lo,
+                               const int32_t* perm, const float* lse, float* D, float* dqk,
+                               float* dv, void* ws, int* status, cudaStream_t s) {
   if (!tc_eligible(p)) return cudaErrorNotSupported;
   const TcWs w = tc_ws(p, ws);
   const int n_chunks = p.L / kM;
@@ -774,6 +819,9 @@ cudaError_t launch_attn_bwd_tc(const lsh_problem& p, const void* qk, const void*
       !encode_tmap_2d_16bit(&m_dqk, w.part_dqk, 64, (uint64_t)rows, 128, 64, 64) ||
       !encode_tmap_2d_16bit(&m_edge, w.edge, 64, (uint64_t)(n_units * kM), 128, 64, 64))
     return cudaErrorInvalidValue;
+  bwd_prep_tc_kernel<<<(unsigned)((N * 8 + 255) / 256), 256, 0, s>>>(
+      (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, (const __nv_bfloat16*)dout,
+      (const __nv_bfloat16*)out, (const __nv_bfloat16*)out_lo, D, w.x16, w.v16, w.g16, N);
   inverse_perm_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(perm, w.inv, p.L, rows,
                                                                       status);
   int grid = sm_count();
@@ -783,13 +831,13 @@ cudaError_t launch_attn_bwd_tc(const lsh_problem& p, const void* qk, const void*
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemBytes, s>>>(
-      (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, (const __nv_bfloat16*)dout, perm, lse, D,
+      w.x16, w.v16, w.g16, perm, lse, D,
       m_dv, m_dqk, m_edge, p.L, p.n_rounds, p.scale, p.scale * kLog2e, (int)n_units,
       units_per_seg, status);
   unsort_kernel<<<(unsigned)((N * 8 + 255) / 256), 256, 0, s>>>(
       w.part_dv, w.part_dqk, w.edge, w.inv, lse, (const __nv_bfloat16*)dout, dqk, dv, p.L,
       p.n_rounds, units_per_seg, N, status);
-  note_launch(3);
+  note_launch(4);
   return cudaGetLastError();
 }
 
