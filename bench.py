@@ -25,7 +25,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from efficient_transformer_lsh_b200.workloads import HEADLINE, WORKLOADS, generate  # noqa: E402
+from efficient_transformer_lsh_b200.workloads import (HEADLINE, WORKLOADS, generate,  # noqa: E402
+                                                      generate_slices)
 
 METRIC = "LSH-attn fwd+bwd tokens/s at L=64K, 8 heads, 4 rounds; % of roofline"
 UNIT = "tokens/s"
@@ -134,74 +135,124 @@ class ClockSampler:
 # CPU oracle timing (baseline leg and the reference arm)
 # ----------------------------------------------------------------------------
 
-def oracle_sample_step(w, inp64, heads):
-    """hash + sort + forward (+ backward) of the oracle on `heads` (b=0) slices at full L."""
-    from oracle import lsh_oracle as orc
-    qk = inp64["qk"][:1, :heads]
-    v = inp64["v"][:1, :heads]
-    bucket, _ = orc.hash_buckets(qk, inp64["R"])
-    perm = orc.sort_positions(bucket)
-    O, LSE = orc.forward(qk, v, perm, w.chunk, w.causal, w.scale)
-    if w.backward:
-        orc.backward(qk, v, perm, w.chunk, w.causal, w.scale, O, LSE, inp64["dO"][:1, :heads])
-
-
-def oracle_threads():
+def _pool_init():
+    # one BLAS thread per worker process: the pool's size is the core count used
     try:
-        from threadpoolctl import threadpool_info
-        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
     except Exception:
-        n = 1
-    return int(n)
+        pass
 
 
-def oracle_inputs(w):
+def _oracle_slice(task):
+    """hash + sort + forward (+ backward) of the oracle on one (batch, head)
+    slice at full L (runs in a pool worker)."""
     import numpy as np
-    inp = generate(w.with_sizes(B=1))
-    return {k: a.astype(np.float64) for k, a in inp.items()}
+    from oracle import lsh_oracle as orc
+    qk, v, dO, R, chunk, causal, scale, backward = task
+    qk = qk.astype(np.float64)[None, None]
+    v = v.astype(np.float64)[None, None]
+    bucket, _ = orc.hash_buckets(qk, R.astype(np.float64))
+    perm = orc.sort_positions(bucket)
+    O, LSE = orc.forward(qk, v, perm, chunk, causal, scale)
+    if backward:
+        orc.backward(qk, v, perm, chunk, causal, scale, O, LSE, dO.astype(np.float64)[None, None])
+    return True
 
 
-def cpu_baseline(w, heads):
-    inp64 = oracle_inputs(w)
-    t = time.perf_counter()
-    oracle_sample_step(w, inp64, heads)
-    dt = time.perf_counter() - t
-    frac = heads / (w.B * w.H)
-    return {"value": w.tokens * frac / dt, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-            "seconds": dt,
-            "sample": f"{heads} of {w.B * w.H} (batch, head) slices at full L={w.L}, all "
-                      f"{w.n_rounds} rounds, hash+sort+fwd{'+bwd' if w.backward else ''}; "
-                      f"tokens/s scaled by the slice fraction {frac:.4f}"}
+class OracleTimer:
+    """Times the float64 oracle on the host cores: one (batch, head) slice per
+    worker of a spawn-started process pool, all slices at once."""
+
+    def __init__(self, w):
+        import multiprocessing as mp
+        self.w = w
+        inp = generate(w)
+        n_slices = w.B * w.H
+        self.cores = max(1, min(n_slices, len(os.sched_getaffinity(0))))
+        self.tasks = []
+        for k in range(self.cores):
+            b, h = divmod(k, w.H)
+            dO = inp["dO"][b, h] if w.backward else None
+            self.tasks.append((inp["qk"][b, h], inp["v"][b, h], dO, inp["R"], w.chunk, w.causal,
+                               w.scale, w.backward))
+        self.frac = self.cores / n_slices
+        self.pool = mp.get_context("spawn").Pool(self.cores, initializer=_pool_init)
+
+    def run(self):
+        t = time.perf_counter()
+        self.pool.map(_oracle_slice, self.tasks, chunksize=1)
+        return time.perf_counter() - t
+
+    def sample(self):
+        w = self.w
+        return (f"{self.cores} of {w.B * w.H} (batch, head) slices at full L={w.L}, one per worker "
+                f"process, all {w.n_rounds} rounds, hash+sort+fwd{'+bwd' if w.backward else ''}; "
+                f"tokens/s scaled by the slice fraction {self.frac:.4f}")
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def cpu_baseline(w):
+    timer = OracleTimer(w)
+    try:
+        timer.run()                      # workers start and import numpy
+        dt = timer.run()
+    finally:
+        timer.close()
+    return {"value": w.tokens * timer.frac / dt, "unit": UNIT, "cores": timer.cores,
+            "kind": "oracle", "seconds": dt, "sample": timer.sample()}
 
 
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", 0))
     if rank != 0:
         return 0
-    inp64 = oracle_inputs(w)
-    heads = 1
-    for _ in range(args.warmup):
-        oracle_sample_step(w, inp64, heads)
-    times = []
-    for _ in range(args.steps):
-        t = time.perf_counter()
-        oracle_sample_step(w, inp64, heads)
-        times.append(time.perf_counter() - t)
-    frac = heads / (w.B * w.H)
+    timer = OracleTimer(w)
+    try:
+        for _ in range(args.warmup):
+            timer.run()
+        times = [timer.run() for _ in range(args.steps)]
+    finally:
+        timer.close()
     per_step = sum(times) / len(times)
-    value = w.tokens * frac / per_step
+    value = w.tokens * timer.frac / per_step
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3 / frac,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3 / timer.frac,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(w),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-                         "sample": f"each step: {heads} of {w.B * w.H} (batch, head) slices at full "
-                                   f"L={w.L}; tokens/s scaled by {frac:.4f}"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": timer.cores, "kind": "oracle",
+                         "sample": "each step: " + timer.sample()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def source_digest(files):
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload, stage):
+    """DRAM bytes per launch of a stage's kernels from the committed ncu
+    summary (profiles/traffic.json), or None when there is none or when the
+    kernel sources changed since the counters were taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            e = json.load(f).get(workload, {}).get(stage)
+        if not e or source_digest(e["sources"]) != e["digest"]:
+            return None
+        return e["bytes"]
+    except Exception:
+        return None
 
 
 def config_of(w):
@@ -221,11 +272,17 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS))
-    ap.add_argument("--cpu-heads", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override H (smaller cases of the same kernels, e.g. for profiler captures)")
+    ap.add_argument("--seq-len", type=int, default=None, help="override L")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
+    if args.heads is not None:
+        w = w.with_sizes(H=args.heads)
+    if args.seq_len is not None:
+        w = w.with_sizes(L=args.seq_len)
     if args.impl == "reference":
         return run_reference(args, w)
     args.warmup = max(3, args.warmup)
@@ -243,8 +300,14 @@ def main():
     torch.cuda.set_device(dev)
     _lib.lib()
 
-    seed = dist.rank_seed(20200 + w.index, rank)
-    inp = generate(w, seed=seed)
+    # one global problem of world x B batches; this rank runs its shard of
+    # B*H slices (weak scaling: the per-rank work is fixed)
+    gw = w.with_sizes(B=w.B * world)
+    lo, hi = dist.shard(gw.B * gw.H, rank, world)
+    inp = generate_slices(gw, lo, hi)
+    for k in ("qk", "v", "dO"):
+        if k in inp:
+            inp[k] = inp[k].reshape(w.B, w.H, w.L, w.d)
     td = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     host = {k: torch.from_numpy(a).to(td).pin_memory() for k, a in inp.items()}
     d_in = {k: t.to(dev, non_blocking=True) for k, t in host.items()}
@@ -270,10 +333,16 @@ def main():
             if evs is not None:
                 evs[4].record(stream)
 
+    torch.cuda.synchronize(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
     assert _lib.lsh_device_status(stream) == 0
+    memory = {"peak_bytes": int(torch.cuda.max_memory_allocated(dev)),
+              "workspace_bytes": int(run.ws_sort_bytes + run.ws_fwd_bytes + run.ws_bwd_bytes),
+              "note": "device memory torch allocated for one problem: inputs, outputs, "
+                      "bucket/perm and the three workspaces"}
 
     # timed region: K whole steps, device time, max over ranks
     gpu_index = os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local if world > 1 else 0]
@@ -321,16 +390,7 @@ def main():
                      "frac": max(t_b, t_f) / t}
     dom = max(names, key=lambda n: stage_ms[n])
     ds = stages[dom]
-    traffic = None
-    tr_file = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tr_file):
-        try:
-            with open(tr_file) as f:
-                tr = json.load(f).get(w.name, {}).get(dom)
-            if tr is not None:
-                traffic = tr
-        except Exception:
-            traffic = None
+    traffic = measured_traffic(w.name, dom)
     if ds["bound"] == "hbm":
         roof = {"bound": "hbm", "achieved": ds["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     else:
@@ -380,9 +440,10 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": config_of(w), "roofline": roof, "step_roofline": step_roof, "stages": stages,
         "e2e": e2e, "gpu_launches": launches, "clocks": sampler.summary(t_host0, t_host1),
+        "memory": memory,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, min(args.cpu_heads, w.B * w.H))
+        line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
         print(json.dumps(line), flush=True)
     dist.finish()

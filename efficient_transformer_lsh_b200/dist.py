@@ -1,9 +1,12 @@
-"""Multi-process plumbing: one process per GPU, independent problems per rank.
+"""Multi-process plumbing: one process per GPU, one shard of a problem per rank.
 
 Every (batch, head) slice of LSH attention is independent through hashing,
-sorting, chunk attention, the round combine and the backward pass, so ranks
-share no data: each rank runs its own problem (weak scaling) and the only
-collective is the max-over-ranks reduction of the measured time.
+sorting, chunk attention, the round combine and the backward pass, so a
+problem is split across ranks by contiguous ranges of its B*H slices
+(``shard``) and each rank runs its range through the C ABI as a problem of
+its own (the slices are contiguous in the [B, H, L, d] layout). Ranks share
+no data; the only collective is the max-over-ranks reduction of the
+measured time.
 """
 from __future__ import annotations
 
@@ -28,11 +31,6 @@ def init(backend: str, timeout_s: float = 120.0) -> Tuple[int, int, int]:
         dist.init_process_group(backend, rank=rank, world_size=world,
                                 timeout=datetime.timedelta(seconds=timeout_s))
     return rank, local, world
-
-
-def rank_seed(base: int, rank: int) -> int:
-    """Seed of rank ``rank``'s independent problem (rank 0 keeps ``base``)."""
-    return base + 7919 * rank
 
 
 def shard(n: int, rank: int, world: int) -> Tuple[int, int]:

@@ -5,16 +5,21 @@ It holds none of the attention arithmetic, so the CUDA path and the CPU
 oracle can both take their inputs from it without sharing any of the method.
 
 Recipe (one per named workload):
-  * generator: numpy PCG64 seeded with ``20200 + index``; ``SeedSequence.spawn``
-    gives independent streams for qk, v, R and dO;
+  * generator: numpy PCG64; every array of every (batch, head) slice has its
+    own stream, seeded by SeedSequence([seed, array id, slice index]) with
+    ``seed = 20200 + index``, so any contiguous range of slices (one rank's
+    shard of a problem) can be drawn on its own and equals the same slices
+    of the whole problem; R and the mixture's cluster centres have streams
+    of their own;
   * values are drawn in float64 and rounded once to the input dtype
     (round-to-nearest-even); bf16 values are returned as float32 arrays whose
     values are exactly representable in bf16, so widening them is exact;
   * qk, v, dO have shape [B, H, L, d]; R has shape [n_rounds, d, n_buckets/2]
     (one random rotation per hash round, shared by every batch and head);
-  * ``qk="mixture"`` draws 256 cluster centres ~ N(0, I) and gives every token
-    a uniformly chosen centre plus N(0, 0.1^2) noise, which makes bucket
-    occupancy uneven the way real text does; every other array is N(0, 1).
+  * ``qk="mixture"`` draws 256 cluster centres ~ N(0, I) (shared by all
+    slices) and gives every token a uniformly chosen centre plus
+    N(0, 0.1^2) noise, which makes bucket occupancy uneven the way real text
+    does; every other array is N(0, 1).
 
 The sizes mirror the experiments named on the Reformer pages (64K-token
 enwik8, 12K-token imagenet-64, half-million-token sequences); the datasets
@@ -108,34 +113,57 @@ def _to_dtype(a: np.ndarray, dtype: str) -> np.ndarray:
     raise ValueError(dtype)
 
 
+_QK, _V, _DO, _R, _CENTRES = 0, 1, 2, 3, 4
+
+
+def _stream(seed: int, array: int, k: int = 0) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, array, k])))
+
+
+def generate_slices(w: Workload, lo: int, hi: int, seed: Optional[int] = None,
+                    with_grad: Optional[bool] = None):
+    """Draw the (batch, head) slices [lo, hi) of workload ``w`` (flattened
+    index b * H + h). Returns qk, v (and dO) of shape [hi - lo, L, d] and R."""
+    if seed is None:
+        seed = 20200 + w.index
+    if with_grad is None:
+        with_grad = w.backward
+    n = hi - lo
+    shape = (n, w.L, w.d)
+    out = {}
+    if w.qk == "mixture":
+        centres = _stream(seed, _CENTRES).standard_normal((w.n_clusters, w.d))
+    qk = np.empty(shape)
+    for i, k in enumerate(range(lo, hi)):
+        g = _stream(seed, _QK, k)
+        if w.qk == "mixture":
+            assign = g.integers(0, w.n_clusters, size=w.L)
+            qk[i] = centres[assign] + w.cluster_sigma * g.standard_normal((w.L, w.d))
+        elif w.qk == "normal":
+            qk[i] = g.standard_normal((w.L, w.d))
+        else:
+            raise ValueError(w.qk)
+    out["qk"] = _to_dtype(qk, w.dtype)
+    del qk
+    out["v"] = _to_dtype(np.stack([_stream(seed, _V, k).standard_normal((w.L, w.d))
+                                   for k in range(lo, hi)]) if n else np.empty(shape), w.dtype)
+    out["R"] = _to_dtype(_stream(seed, _R).standard_normal((w.n_rounds, w.d, w.n_buckets // 2)),
+                         w.dtype)
+    if with_grad:
+        out["dO"] = _to_dtype(np.stack([_stream(seed, _DO, k).standard_normal((w.L, w.d))
+                                        for k in range(lo, hi)]) if n else np.empty(shape),
+                              w.dtype)
+    return out
+
+
 def generate(w: Workload, seed: Optional[int] = None, with_grad: Optional[bool] = None):
     """Draw the inputs of workload ``w``.
 
     Returns a dict of float32 numpy arrays: qk, v, R and (when a backward pass
     is wanted) dO. Values are exactly representable in ``w.dtype``.
     """
-    if seed is None:
-        seed = 20200 + w.index
-    if with_grad is None:
-        with_grad = w.backward
-    s_qk, s_v, s_r, s_do = np.random.SeedSequence(seed).spawn(4)
-    shape = (w.B, w.H, w.L, w.d)
-    g = np.random.Generator(np.random.PCG64(s_qk))
-    if w.qk == "mixture":
-        centres = g.standard_normal((w.n_clusters, w.d))
-        assign = g.integers(0, w.n_clusters, size=shape[:-1])
-        qk = centres[assign] + w.cluster_sigma * g.standard_normal(shape)
-    elif w.qk == "normal":
-        qk = g.standard_normal(shape)
-    else:
-        raise ValueError(w.qk)
-    out = {"qk": _to_dtype(qk, w.dtype)}
-    del qk
-    out["v"] = _to_dtype(np.random.Generator(np.random.PCG64(s_v)).standard_normal(shape), w.dtype)
-    out["R"] = _to_dtype(
-        np.random.Generator(np.random.PCG64(s_r)).standard_normal(
-            (w.n_rounds, w.d, w.n_buckets // 2)), w.dtype)
-    if with_grad:
-        out["dO"] = _to_dtype(
-            np.random.Generator(np.random.PCG64(s_do)).standard_normal(shape), w.dtype)
+    out = generate_slices(w, 0, w.B * w.H, seed, with_grad)
+    for k in ("qk", "v", "dO"):
+        if k in out:
+            out[k] = out[k].reshape(w.B, w.H, w.L, w.d)
     return out

@@ -1,8 +1,9 @@
 """Multi-process plumbing on CPU: two gloo ranks, no GPU.
 
-Each rank runs an independent problem (weak scaling): seeds differ per rank,
-(batch, head) slices partition exactly, and the reported time is the max
-over ranks."""
+A problem is split across ranks by contiguous ranges of its (batch, head)
+slices; each rank draws and runs only its shard, and the reported time is
+the max over ranks. Running the oracle shard by shard on the ranks gives
+exactly the whole problem's result (the slices are independent)."""
 import os
 import socket
 
@@ -26,11 +27,17 @@ def _worker(rank, world, port, q):
     t = dist.max_over_ranks(1.5 + rank)          # rank 1 is the slower one
     lo, hi = dist.shard(13, r, w)
     import numpy as np
-    from efficient_transformer_lsh_b200.workloads import WORKLOADS, generate
-    wl = WORKLOADS["toy-f32-L1024"].with_sizes(L=128)
-    x = generate(wl, seed=dist.rank_seed(100, r))["qk"]
+    from efficient_transformer_lsh_b200.workloads import WORKLOADS, generate_slices
+    from oracle import lsh_oracle as orc
+    # one global problem of 2 x 3 slices; this rank's shard through the oracle
+    gw = WORKLOADS["batch-bf16-8x8x4096"].with_sizes(B=2, H=3, L=256, n_rounds=2)
+    s0, s1 = dist.shard(gw.B * gw.H, r, w)
+    inp = generate_slices(gw, s0, s1)
+    qk = inp["qk"].astype(np.float64)[None]
+    v = inp["v"].astype(np.float64)[None]
+    res = orc.lsh_attention(qk, v, inp["R"].astype(np.float64), gw.chunk, gw.causal, gw.scale)
     gathered = [None] * w
-    torch.distributed.all_gather_object(gathered, (lo, hi, float(np.asarray(x).sum())))
+    torch.distributed.all_gather_object(gathered, (lo, hi, s0, s1, res["O"][0], res["LSE"][0]))
     dist.barrier()
     dist.finish()
     q.put((r, t, gathered))
@@ -47,11 +54,23 @@ def test_two_gloo_ranks():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
+    import numpy as np
+    from efficient_transformer_lsh_b200.workloads import WORKLOADS, generate
+    from oracle import lsh_oracle as orc
+    gw = WORKLOADS["batch-bf16-8x8x4096"].with_sizes(B=2, H=3, L=256, n_rounds=2)
+    whole = generate(gw)
+    full = orc.lsh_attention(whole["qk"].astype(np.float64), whole["v"].astype(np.float64),
+                             whole["R"].astype(np.float64), gw.chunk, gw.causal, gw.scale)
     for r, t, gathered in res:
         assert t == 2.5                      # max over ranks
-        (lo0, hi0, s0), (lo1, hi1, s1) = gathered
+        (lo0, hi0, a0, b0, O0, L0), (lo1, hi1, a1, b1, O1, L1) = gathered
         assert (lo0, hi0, lo1, hi1) == (0, 7, 7, 13)
-        assert s0 != s1                      # independent problems per rank
+        assert (a0, b0, a1, b1) == (0, 3, 3, 6)
+        # the shards' results, put together, are the whole problem's
+        O = np.concatenate([O0, O1]).reshape(full["O"].shape)
+        LSE = np.concatenate([L0, L1]).reshape(full["LSE"].shape)
+        np.testing.assert_array_equal(O, full["O"])
+        np.testing.assert_array_equal(LSE, full["LSE"])
 
 
 def test_shard_covers_everything():
