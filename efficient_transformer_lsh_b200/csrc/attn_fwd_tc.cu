@@ -253,7 +253,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
     };
     auto checked = [&](int ps) {
       if ((unsigned)ps >= (unsigned)L) {
-        if (status) atomicExch(status, (int)LSH_ERR_DEVICE_CHECK);
+        record_status(status, (int)LSH_ERR_DEVICE_CHECK);
         ps = 0;
       }
       return ps;
