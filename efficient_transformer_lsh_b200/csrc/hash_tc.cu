@@ -9,24 +9,29 @@
 // products into float32 accumulators in TMEM: this is a float32 contraction
 // of exact products, as on the CUDA-core path.
 //
-// Structure (one CTA per SM, persistent; CTAs are assigned to one round so
-// that R_r stays resident in shared memory):
-//   warp 0  : TMA producer — R_r once (MN-major operand), then 128-token X
-//             tiles (K-major) through a 4-stage ring, released by the MMAs;
+// Structure (one CTA per SM, persistent; CTAs are assigned to one round):
+//   warp 0  : TMA producer — 128-token X tiles (K-major) through a 4-stage
+//             ring, released by the MMAs; R_r as 512-column blocks of the
+//             MN-major operand: one block stays resident when n_b/2 <= 512,
+//             otherwise the blocks stream through a 2-stage ring, once per
+//             pair of X tiles (both tiles use each block);
 //   warp 1  : TMEM allocation; one thread issues tcgen05.mma: a 128 x 256 x 64
-//             product per 256-column chunk of R_r;
+//             product per 256-column chunk of a block, the chunks of a pair
+//             of tiles interleaved;
 //   warps 2-5, 6-9: two epilogue warpgroups taking alternate tiles, each with
 //             its own 256-column TMEM accumulator (one token per thread).
-//             Each s becomes a float key whose 4 low mantissa bits hold
-//             (15 - its 32-column group) and whose sign is kept; two 3-input
-//             max and min operations fold two columns into each of 32
-//             per-position running maxima (largest +s) and minima (most
-//             negative s), the lowest column winning ties. Values closer than
-//             2^-19 relative count as ties (a near-tie by the 1e-5 bound the
-//             results are checked against). The merge picks the larger of the
-//             best +s and the best -s, the +s half first on ties.
-// Handles n_b/2 <= 512 with n_b/2 a multiple of 8; other shapes use the
-// CUDA-core kernel.
+//             Each s becomes a float key whose 6 low mantissa bits hold
+//             (63 - its column / 8 within the block) and whose sign is kept;
+//             two 3-input max and min operations fold two columns into each
+//             of 8 running maxima (largest +s) and minima (most negative s),
+//             one per column mod 8. Keys keep 17 mantissa bits, so values
+//             2^-17 (7.6e-6) relative apart still order correctly: equal keys
+//             are a near-tie by the 1e-5 bound the results are checked
+//             against. After each block the 8 slots are merged into the
+//             running best (largest |s|; on ties the +s half, then the lower
+//             column).
+// Handles n_b/2 a multiple of 8 up to 32768; other shapes use the CUDA-core
+// kernel.
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
@@ -39,15 +44,17 @@ using namespace tc;
 
 constexpr int kTileM = 128;          // tokens per tile
 constexpr int kStages = 4;           // X ring depth
-constexpr int kMaxNh = 512;          // rotation columns resident per round
+constexpr int kBlockN = 512;         // rotation columns per R block
 constexpr int kChunkN = 256;         // columns per MMA / accumulator
-constexpr int kXBytes = kTileM * 128;              // 16 KB
-constexpr int kRBlockBytes = 64 * 128;             // 64 columns x 64 k-rows
-constexpr int kRBytes = (kMaxNh / 64) * kRBlockBytes;  // 64 KB
+constexpr int kRStages = 2;          // R ring depth when R is streamed
+constexpr int kXBytes = kTileM * 128;                    // 16 KB
+constexpr int kRBoxBytes = 64 * 128;                     // 64 columns x 64 k-rows
+constexpr int kRBlockBytes = (kBlockN / 64) * kRBoxBytes;  // 64 KB
 constexpr int kThreads = 320;
 
 struct __align__(8) HashBarriers {
-  uint64_t r_full;
+  uint64_t r_full[kRStages];
+  uint64_t r_empty[kRStages];
   uint64_t x_full[kStages];
   uint64_t x_empty[kStages];
   uint64_t acc_full[2];
@@ -57,22 +64,28 @@ struct __align__(8) HashBarriers {
   int abort;
 };
 
-constexpr size_t kSmemBytes = 1024 + kRBytes + kStages * kXBytes + sizeof(HashBarriers);
+constexpr size_t kSmemBytes =
+    1024 + kRStages * kRBlockBytes + kStages * kXBytes + sizeof(HashBarriers);
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
-// Folds two accumulator values (raw fp32 bits a, b; group tags ta, tb in the
-// low 4 mantissa bits) into the running maximum and minimum of one position.
+// Folds two accumulator values (raw fp32 bits a, b) into the running maximum
+// and minimum of one slot, after replacing their 6 low mantissa bits by their
+// tags ta, tb (63 - column / 8 within the R block).
 __device__ __forceinline__ void fold2(float& mx, float& mn, uint32_t a, uint32_t b, uint32_t ta,
                                       uint32_t tb) {
-  const float ka = __uint_as_float((a & 0xFFFFFFF0u) | ta);
-  const float kb = __uint_as_float((b & 0xFFFFFFF0u) | tb);
+  const float ka = __uint_as_float((a & 0xFFFFFFC0u) | ta);
+  const float kb = __uint_as_float((b & 0xFFFFFFC0u) | tb);
   float r0, r1;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r0) : "f"(mx), "f"(ka), "f"(kb));
   asm("min.f32 %0, %1, %2, %3;" : "=f"(r1) : "f"(mn), "f"(ka), "f"(kb));
   mx = r0;
   mn = r1;
 }
+
+// Columns of R block b: [512 b, min(nh, 512 b + 512)).
+__device__ __forceinline__ int block_cols(int nh, int b) { return min(kBlockN, nh - b * kBlockN); }
 
 __global__ void __launch_bounds__(kThreads, 1)
 hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_r,
@@ -81,21 +94,27 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* r_smem = smem;
-  uint8_t* x_smem = smem + kRBytes;
+  uint8_t* x_smem = smem + kRStages * kRBlockBytes;
   HashBarriers* bar = (HashBarriers*)(x_smem + kStages * kXBytes);
   volatile int* abort = &bar->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x % n_rounds;
   const int ci = blockIdx.x / n_rounds;
-  const int n_blk = (nh + 63) / 64;
-  const int nsub = (nh + kChunkN - 1) / kChunkN;
+  const int n_blk = (nh + kBlockN - 1) / kBlockN;
+  // one R block stays resident; several are streamed through the R ring,
+  // once per pair of tiles
+  const bool stream_r = n_blk > 1;
+  const int n_mine = ci < n_tiles ? (n_tiles - ci + ctas_per_round - 1) / ctas_per_round : 0;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bar->r_full, 1);
+    for (int s = 0; s < kRStages; ++s) {
+      mbar_init(&bar->r_full[s], 1);
+      mbar_init(&bar->r_empty[s], 1);     // released by the MMAs' commit
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar->x_full[s], 1);
-      mbar_init(&bar->x_empty[s], 1);     // released by the MMAs' commit
+      mbar_init(&bar->x_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar->acc_full[b], 1);
@@ -119,46 +138,87 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
       // ---------------- producer ----------------
       prefetch_tmap(&map_x);
       prefetch_tmap(&map_r);
-      mbar_expect_tx(&bar->r_full, n_blk * kRBlockBytes);
-      for (int b = 0; b < n_blk; ++b)
-        tma_load_2d(r_smem + b * kRBlockBytes, &map_r, b * 64, r * 64, &bar->r_full);
-      int it = 0;
-      for (int t = ci; t < n_tiles; t += ctas_per_round, ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-        if (it >= kStages && !mbar_wait(&bar->x_empty[s], ph ^ 1u, abort, status)) break;
-        mbar_expect_tx(&bar->x_full[s], kXBytes);
-        tma_load_2d(x_smem + s * kXBytes, &map_x, 0, t * kTileM, &bar->x_full[s]);
+      // R block b into ring stage rs
+      auto load_r = [&](int b, int rs) {
+        const int nbox = (block_cols(nh, b) + 63) / 64;
+        mbar_expect_tx(&bar->r_full[rs], nbox * kRBoxBytes);
+        for (int k = 0; k < nbox; ++k)
+          tma_load_2d(r_smem + rs * kRBlockBytes + k * kRBoxBytes, &map_r, b * kBlockN + k * 64,
+                      r * 64, &bar->r_full[rs]);
+      };
+      int rb = 0;                            // R blocks loaded
+      if (!stream_r) {
+        load_r(0, 0);
+        rb = 1;
+      }
+      int it = 0;                            // X tiles loaded
+      bool ok = true;
+      for (int it0 = 0; it0 < n_mine && ok; it0 += 2) {
+        const int cnt = min(2, n_mine - it0);
+        for (int k = 0; k < cnt && ok; ++k, ++it) {
+          const int s = it % kStages;
+          if (it >= kStages &&
+              !mbar_wait(&bar->x_empty[s], (uint32_t)(it / kStages - 1) & 1u, abort, status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&bar->x_full[s], kXBytes);
+          tma_load_2d(x_smem + s * kXBytes, &map_x, 0, (ci + it * ctas_per_round) * kTileM,
+                      &bar->x_full[s]);
+        }
+        if (stream_r) {
+          for (int b = 0; b < n_blk && ok; ++b, ++rb) {
+            const int rs = rb % kRStages;
+            if (rb >= kRStages &&
+                !mbar_wait(&bar->r_empty[rs], (uint32_t)(rb / kRStages - 1) & 1u, abort, status)) {
+              ok = false;
+              break;
+            }
+            load_r(b, rs);
+          }
+        }
       }
       // every issued copy has landed before the CTA may exit (bounded)
-      const int issued = it;
-      for (int s = 0; s < kStages && s < issued; ++s) {
-        const int last = issued - 1 - ((issued - 1 - s) % kStages);
-        int dummy = 0;
+      int dummy = 0;
+      for (int s = 0; s < kStages && s < it; ++s) {
+        const int last = it - 1 - ((it - 1 - s) % kStages);
         mbar_wait(&bar->x_full[s], (uint32_t)(last / kStages) & 1u, (volatile int*)&dummy, status);
       }
-      int dummy = 0;
-      mbar_wait(&bar->r_full, 0, (volatile int*)&dummy, status);
+      for (int s = 0; s < kRStages && s < rb; ++s) {
+        const int last = rb - 1 - ((rb - 1 - s) % kRStages);
+        mbar_wait(&bar->r_full[s], (uint32_t)(last / kRStages) & 1u, (volatile int*)&dummy, status);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
       // Tiles alternate between the two accumulators / epilogue warpgroups;
-      // the chunks of a pair of tiles are interleaved so both stay busy.
-      if (mbar_wait(&bar->r_full, 0, abort, status)) {
+      // the chunks of a pair of tiles are interleaved so both stay busy, and
+      // a streamed R block serves both tiles of the pair.
+      const uint32_t r_lo = (smem_u32(r_smem) >> 4) | desc_lbo(kRBoxBytes);
+      const uint32_t x_lo = (smem_u32(x_smem) >> 4) | desc_lbo(16);
+      int uses0 = 0, uses1 = 0, rb = 0;
+      bool ok = true;
+      if (!stream_r) {
+        ok = mbar_wait(&bar->r_full[0], 0u, abort, status);
+        rb = 1;
+      }
+      for (int it0 = 0; it0 < n_mine && ok; it0 += 2) {
+        const int cnt = min(2, n_mine - it0);
+        for (int k = 0; k < cnt && ok; ++k)
+          ok = mbar_wait(&bar->x_full[(it0 + k) % kStages], (uint32_t)((it0 + k) / kStages) & 1u,
+                         abort, status);
+        if (!ok) break;
         tc_fence_after();
-        const uint32_t r_lo = (smem_u32(r_smem) >> 4) | desc_lbo(kRBlockBytes);
-        const uint32_t x_lo = (smem_u32(x_smem) >> 4) | desc_lbo(16);
-        int uses0 = 0, uses1 = 0;
-        bool ok = true;
-        const int n_mine = (n_tiles - ci + ctas_per_round - 1) / ctas_per_round;
-        for (int it0 = 0; it0 < n_mine && ok; it0 += 2) {
-          const int cnt = min(2, n_mine - it0);
-          for (int k = 0; k < cnt && ok; ++k)
-            ok = mbar_wait(&bar->x_full[(it0 + k) % kStages],
-                           (uint32_t)((it0 + k) / kStages) & 1u, abort, status);
-          if (!ok) break;
-          tc_fence_after();
+        for (int b = 0; b < n_blk && ok; ++b) {
+          const int rs = stream_r ? rb % kRStages : 0;
+          if (stream_r) {
+            ok = mbar_wait(&bar->r_full[rs], (uint32_t)(rb / kRStages) & 1u, abort, status);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          const int bcols = block_cols(nh, b);
+          const int nsub = (bcols + kChunkN - 1) / kChunkN;
           for (int j = 0; j < nsub && ok; ++j)
             for (int k = 0; k < cnt && ok; ++k) {
               const int it = it0 + k, w = it & 1, s = it % kStages;
@@ -170,20 +230,25 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
               }
               ++uses;
               tc_fence_after();
-              const int ncols = min(kChunkN, nh - j * kChunkN);
-              // whole 64-column blocks: the MN-major operand is read in complete
+              const int ncols = min(kChunkN, bcols - j * kChunkN);
+              // whole 64-column boxes: the MN-major operand is read in complete
               // swizzle atoms; the zero-filled extra columns are masked later
               const int n_mma = (ncols + 63) / 64 * 64;
               const uint32_t idesc = idesc_f16(kTileM, n_mma, 1, false, true);
               const uint32_t d = tmem + (uint32_t)(w * kChunkN);
               const uint32_t a = x_lo + (uint32_t)(s * kXBytes) / 16;
-              const uint32_t b = r_lo + (uint32_t)(j * 4 * kRBlockBytes) / 16;
+              const uint32_t bd =
+                  r_lo + (uint32_t)(rs * kRBlockBytes + j * 4 * kRBoxBytes) / 16;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                mma_ss_w(d, a + 2 * kk, b + 128 * kk, kDescHi1024, idesc, kk > 0);
+                mma_ss_w(d, a + 2 * kk, bd + 128 * kk, kDescHi1024, idesc, kk > 0);
               mma_commit(&bar->acc_full[w]);
-              if (j == nsub - 1) mma_commit(&bar->x_empty[s]);
+              if (b == n_blk - 1 && j == nsub - 1) mma_commit(&bar->x_empty[s]);
             }
+          if (stream_r && ok) {
+            mma_commit(&bar->r_empty[rs]);
+            ++rb;
+          }
         }
       }
       // all issued MMAs have finished before TMEM is released (bounded)
@@ -197,65 +262,85 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     const int q = warp & 3;                 // TMEM lane quarter this warp may read
     const int row_in_tile = q * 32 + lane;
     const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(w * kChunkN);
-    int use = 0, it = 0;
+    int use = 0;
     bool ok = true;
-    for (int t = ci; t < n_tiles && ok; t += ctas_per_round, ++it) {
-      if ((it & 1) != w) continue;
-      float mx[32], mn[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        mx[i] = -INFINITY;
-        mn[i] = INFINITY;
-      }
-      int g = 0;                              // global 32-column group index
-      for (int j = 0; j < nsub; ++j, ++use) {
-        if (!warp_all(mbar_wait(&bar->acc_full[w], (uint32_t)use & 1u, abort, status))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int ncols = min(kChunkN, nh - j * kChunkN);
-        for (int c0 = 0; c0 < ncols; c0 += 64, g += 2) {
-          uint32_t va[32], vb[32];
-          tmem_ld32(tbase + c0, va);
-          tmem_ld32(tbase + c0 + 32, vb);     // within the accumulator's 256 columns
-          tmem_ld_wait();
-          const uint32_t ma = (uint32_t)(15 - g), mb = (uint32_t)(14 - g);
-          if (ncols - c0 >= 64) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) fold2(mx[i], mn[i], va[i], vb[i], ma, mb);
-          } else {
-            const int na = ncols - c0, nb = ncols - c0 - 32;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              // a missing column is a NaN key, which max and min ignore
-              const uint32_t a = (i < na) ? va[i] : 0x7FFFFFFFu;
-              const uint32_t b = (i < nb) ? vb[i] : 0x7FFFFFFFu;
-              fold2(mx[i], mn[i], a, b, ma, mb);
-            }
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&bar->acc_empty[w]);
-      }
-      if (!ok) break;
-      // merge: largest |s| over both halves; on ties the +s half, then the
-      // smaller column
+    for (int it = w; it < n_mine && ok; it += 2) {
+      const int t = ci + it * ctas_per_round;
       uint32_t best_m = 0;
       int best_c = 0x7fffffff;
+      for (int b = 0; b < n_blk && ok; ++b) {
+        // 8 running slots (column mod 8); keys keep 17 mantissa bits, so
+        // values 2^-17 (7.6e-6) relative apart still order correctly
+        float mx[8], mn[8];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const uint32_t kp = __float_as_uint(mx[i]), kn = __float_as_uint(mn[i]);
-        // a negative running maximum or a positive running minimum (this
-        // includes the initial -inf / +inf) is never the winner
-        const bool vp = (kp >> 31) == 0u, vq = (kn >> 31) != 0u;
-        const uint32_t mp = vp ? (kp & 0x7FFFFFF0u) : 0u;
-        const int cp = vp ? (15 - (int)(kp & 15u)) * 32 + i : 0x7fffffff;
-        const uint32_t mq = vq ? (kn & 0x7FFFFFF0u) : 0u;
-        const int cq = vq ? nh + (15 - (int)(kn & 15u)) * 32 + i : 0x7fffffff;
-        if (mp > best_m || (mp == best_m && cp < best_c)) { best_m = mp; best_c = cp; }
-        if (mq > best_m || (mq == best_m && cq < best_c)) { best_m = mq; best_c = cq; }
+        for (int k = 0; k < 8; ++k) {
+          mx[k] = -INFINITY;
+          mn[k] = INFINITY;
+        }
+        const int bcols = block_cols(nh, b);
+        const int nsub = (bcols + kChunkN - 1) / kChunkN;
+        for (int j = 0; j < nsub; ++j, ++use) {
+          if (!warp_all(mbar_wait(&bar->acc_full[w], (uint32_t)use & 1u, abort, status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int ncols = min(kChunkN, bcols - j * kChunkN);
+          for (int c0 = 0; c0 < ncols; c0 += 64) {
+            uint32_t va[32], vb[32];
+            tmem_ld32(tbase + c0, va);
+            tmem_ld32(tbase + c0 + 32, vb);     // within the accumulator's 256 columns
+            tmem_ld_wait();
+            // tag of block column c: 63 - c / 8; va holds 4 column octets,
+            // vb the next 4
+            const uint32_t t0 = (uint32_t)(63 - (j * kChunkN + c0) / 8);
+            if (ncols - c0 >= 64) {
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+#pragma unroll
+                for (int o = 0; o < 4; o += 2) {
+                  fold2(mx[k], mn[k], va[8 * o + k], va[8 * o + 8 + k], t0 - o, t0 - o - 1);
+                  fold2(mx[k], mn[k], vb[8 * o + k], vb[8 * o + 8 + k], t0 - 4 - o, t0 - 5 - o);
+                }
+              }
+            } else {
+              const int na = ncols - c0, nb = ncols - c0 - 32;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+#pragma unroll
+                for (int o = 0; o < 4; o += 2) {
+                  // a missing column is a NaN key, which max and min ignore
+                  const uint32_t a0 = (8 * o + k < na) ? va[8 * o + k] : 0x7FFFFFFFu;
+                  const uint32_t a1 = (8 * o + 8 + k < na) ? va[8 * o + 8 + k] : 0x7FFFFFFFu;
+                  const uint32_t b0 = (8 * o + k < nb) ? vb[8 * o + k] : 0x7FFFFFFFu;
+                  const uint32_t b1 = (8 * o + 8 + k < nb) ? vb[8 * o + 8 + k] : 0x7FFFFFFFu;
+                  fold2(mx[k], mn[k], a0, a1, t0 - o, t0 - o - 1);
+                  fold2(mx[k], mn[k], b0, b1, t0 - 4 - o, t0 - 5 - o);
+                }
+              }
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&bar->acc_empty[w]);
+        }
+        if (!ok) break;
+        // merge the block into the running best: largest |s|; on ties the +s
+        // half, then the smaller column
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t kp = __float_as_uint(mx[k]), kn = __float_as_uint(mn[k]);
+          // a negative running maximum or a positive running minimum (this
+          // includes the initial -inf / +inf) is never the winner
+          const bool vp = (kp >> 31) == 0u, vq = (kn >> 31) != 0u;
+          const uint32_t mp = vp ? (kp & 0x7FFFFFC0u) : 0u;
+          const int cp = vp ? b * kBlockN + (63 - (int)(kp & 63u)) * 8 + k : 0x7fffffff;
+          const uint32_t mq = vq ? (kn & 0x7FFFFFC0u) : 0u;
+          const int cq = vq ? nh + b * kBlockN + (63 - (int)(kn & 63u)) * 8 + k : 0x7fffffff;
+          if (mp > best_m || (mp == best_m && cp < best_c)) { best_m = mp; best_c = cp; }
+          if (mq > best_m || (mq == best_m && cq < best_c)) { best_m = mq; best_c = cq; }
+        }
       }
+      if (!ok) break;
       const int64_t row = (int64_t)t * kTileM + row_in_tile;
       if (row < n_rows) {
         const int64_t bh = row / L, pos = row - bh * L;
@@ -276,7 +361,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
 cudaError_t launch_hash_tc(const lsh_problem& p, const void* qk, const void* R, int32_t* bucket,
                            int* status, cudaStream_t s) {
   const int nh = p.n_buckets / 2;
-  if (p.dtype != LSH_BF16 || nh > kMaxNh || nh % 8 != 0 || ((uintptr_t)R % 16) != 0)
+  if (p.dtype != LSH_BF16 || nh % 8 != 0 || nh > 32768 || ((uintptr_t)R % 16) != 0)
     return cudaErrorNotSupported;
   const int64_t n_rows = (int64_t)p.B * p.H * p.L;
   const int64_t n_tiles64 = (n_rows + kTileM - 1) / kTileM;

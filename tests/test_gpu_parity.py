@@ -29,6 +29,11 @@ CASES = {
     "bf16-noncausal-m64": W["batch-bf16-8x8x4096"].with_sizes(B=1, H=3, L=1728, n_rounds=3,
                                                                causal=False, backward=True),
     "enwik8-noncausal-m64": W["enwik8-64k-bf16"].with_sizes(H=2, L=4160, causal=False),
+    # more than 1024 buckets: the rotation is streamed in 512-column blocks;
+    # 1032 leaves a second block of 4 columns
+    "bf16-nb1032": W["batch-bf16-8x8x4096"].with_sizes(B=1, H=2, L=1472, n_buckets=1032),
+    "bf16-nb4096-mixture": W["enwik8-64k-bf16"].with_sizes(H=1, L=8192, n_buckets=4096,
+                                                            n_rounds=2),
     # non-causal, chunk 128, odd chunk count
     "bf16-noncausal-m128": W["batch-bf16-8x8x4096"].with_sizes(B=1, H=3, L=1664, chunk=128,
                                                                 causal=False, backward=True),
@@ -158,7 +163,7 @@ def test_sort_paths_bit_exact(B, H, n_r, L, nb):
     from efficient_transformer_lsh_b200 import _lib
     rng = np.random.default_rng(nb + L)
     bucket = rng.integers(0, nb, size=(B, H, n_r, L), dtype=np.int32)
-    bucket[..., ::7] = rng.integers(0, 3, size=bucket[..., ::7].shape)
+    bucket[..., ::7] = rng.integers(0, min(3, nb), size=bucket[..., ::7].shape)
     p = _lib.make_problem(B, H, L, 64, nb, n_r, 64, True, 0.125, "bf16")
     dev = torch.device("cuda")
     bt = torch.from_numpy(bucket).to(dev)
