@@ -7,16 +7,17 @@
 //
 // Counting sort. Two paths:
 //  * n_buckets <= 8192 (every shape the workloads use): two kernels over
-//    blocks of 8K-32K consecutive positions, one CTA each (see the warp path
-//    below): per-warp counts with __match_any_sync, CTA totals per bucket,
-//    then a scatter kernel that forms the bucket bases itself and places
-//    every position at its slot;
+//    blocks of 8K-32K consecutive positions, one CTA each (see the counting
+//    path below): block totals per bucket from shared-memory atomics, then a
+//    scatter kernel that forms the bucket bases itself and ranks positions
+//    with warp-level bitonic sorts of (bucket, lane) keys;
 //  * larger bucket counts: per 4096-position tile the packed keys
 //    (bucket << 12 | local index) are sorted in shared memory by a bitonic
 //    network; row_scan / bucket_scan form the bases; scatter places them.
-// Ranks follow position order inside a warp (lanes in order, steps in order),
-// across the warps of a block (exclusive prefix of their counts) and across
-// blocks (counts of the blocks before), so the whole sort is stable.
+// Ranks follow position order inside a warp step (the lane breaks ties),
+// across the steps of a warp (in order), across the warps of a block
+// (exclusive prefix of their counts) and across blocks (counts of the blocks
+// before), so the whole sort is stable.
 #include <algorithm>
 
 #include "common.cuh"
@@ -177,17 +178,21 @@ scatter_kernel(const uint32_t* __restrict__ sorted, const int32_t* __restrict__ 
   }
 }
 
-// ---- warp-counting path (n_buckets <= kWarpMaxBuckets) --------------------
+// ---- counting path (n_buckets <= kWarpMaxBuckets) -------------------------
 // A segment is cut into Q blocks of P consecutive positions, one CTA each;
-// warp w of a CTA owns PW consecutive positions of its block and counts them
-// into its own 16-bit counters cnt[w][bucket] with __match_any_sync (one
-// leader lane per distinct bucket of a step updates the counter).
-//   sort_count_kernel:   counts[seg][q][bucket] = CTA totals (every bucket
-//                        written, so no clearing pass is needed);
+// warp w of a CTA owns PW consecutive positions of its block.
+//   sort_count_kernel:   counts[seg][q][bucket] = the block's bucket totals,
+//                        from shared-memory atomics (every bucket written, so
+//                        no clearing pass is needed);
 //   sort_scatter_kernel: bucket bases of the segment (exclusive scan of the
 //                        totals over buckets) plus the counts of the blocks
-//                        before q, the per-warp runs inside the block, then
-//                        every position goes to its slot in position order.
+//                        before q; then each warp takes its positions 32 at a
+//                        time, sorts the 32 (bucket, lane) keys with a warp
+//                        bitonic network so equal buckets form contiguous
+//                        segments in lane order, and ranks each position
+//                        within its segment. A first pass counts per warp, an
+//                        exclusive prefix over warps gives each warp's run, and
+//                        a second pass places every position at its slot.
 constexpr int kWarpMaxBuckets = 8192;
 constexpr int kSortSmemBudget = 200 * 1024;
 
@@ -212,56 +217,81 @@ WarpGeo warp_geo(const lsh_problem& p) {
   return g;
 }
 
-// Counts the buckets of this warp's positions [i0, i0 + PW) of the segment
-// (those below L) into cnt[bucket].
-__device__ __forceinline__ void warp_count(const int32_t* __restrict__ seg_bucket, int64_t i0,
-                                           int PW, int L, int lane, uint16_t* cnt,
-                                           int n_buckets, int* status) {
-  for (int st = 0; st < PW; st += 32) {
-    const int64_t i = i0 + st + lane;
-    uint32_t b = 0xffffffffu;
-    if (i < L) {
-      b = (uint32_t)__ldg(seg_bucket + i);
-      if (b >= (uint32_t)n_buckets) {
-        record_status(status, (int)LSH_ERR_DEVICE_CHECK);
-        b = (uint32_t)n_buckets - 1;
-      }
-    }
-    const uint32_t peers = __match_any_sync(0xffffffffu, b);
-    if (i < L && lane == __ffs(peers) - 1) cnt[b] = (uint16_t)(cnt[b] + __popc(peers));
-    __syncwarp();
+// Bucket of position i of the segment (0xffffffff past the end); an id
+// outside [0, n_buckets) is recorded and replaced by n_buckets - 1.
+__device__ __forceinline__ uint32_t load_bucket(const int32_t* __restrict__ seg_bucket, int64_t i,
+                                                int L, int n_buckets, int* status) {
+  if (i >= L) return 0xffffffffu;
+  uint32_t b = (uint32_t)__ldg(seg_bucket + i);
+  if (b >= (uint32_t)n_buckets) {
+    record_status(status, (int)LSH_ERR_DEVICE_CHECK);
+    b = (uint32_t)n_buckets - 1;
   }
+  return b;
 }
 
-__device__ __forceinline__ void zero_counters(uint16_t* cnt, int n) {
-  uint32_t* c32 = reinterpret_cast<uint32_t*>(cnt);   // n is even
-  for (int i = threadIdx.x; i < n / 2; i += blockDim.x) c32[i] = 0u;
+// Sorts the warp's 32 keys ascending (bitonic network over lanes).
+__device__ __forceinline__ uint32_t warp_sort32(uint32_t key, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint32_t o = __shfl_xor_sync(0xffffffffu, key, j);
+      const bool up = (lane & k) == 0, lower = (lane & j) == 0;
+      key = (lower == up) ? min(key, o) : max(key, o);
+    }
+  }
+  return key;
+}
+
+// One step of 32 positions: after sorting (bucket << 5 | lane) keys, lane k
+// holds sorted entry k: its bucket, the lane (position offset) it came from,
+// its rank among the entries of its bucket, and whether it ends the bucket's
+// segment (then `len` is the segment's length).
+struct StepRank {
+  uint32_t bucket;
+  int src, rank, len;
+  bool live, last;
+};
+__device__ __forceinline__ StepRank rank_step(uint32_t b, int lane) {
+  const uint32_t key = warp_sort32(b == 0xffffffffu ? 0xffffffffu : (b << 5) | (uint32_t)lane, lane);
+  StepRank r;
+  r.live = key != 0xffffffffu;
+  r.bucket = key >> 5;
+  r.src = (int)(key & 31u);
+  const uint32_t prev = __shfl_up_sync(0xffffffffu, r.bucket, 1);
+  const uint32_t next = __shfl_down_sync(0xffffffffu, r.bucket, 1);
+  const bool first = lane == 0 || prev != r.bucket;
+  r.last = lane == 31 || next != r.bucket;
+  const uint32_t starts = __ballot_sync(0xffffffffu, first);
+  const int seg0 = 31 - __clz(starts & (0xffffffffu >> (31 - lane)));
+  r.rank = lane - seg0;
+  r.len = r.rank + 1;
+  return r;
 }
 
 __global__ void __launch_bounds__(1024)
 sort_count_kernel(const int32_t* __restrict__ bucket, int32_t* __restrict__ counts, int L,
-                  int n_buckets, int PW, int P, int Q, int* status) {
+                  int n_buckets, int P, int Q, int* status) {
   extern __shared__ __align__(16) uint8_t sm[];
-  uint16_t* cnt = reinterpret_cast<uint16_t*>(sm);      // [W][n_buckets]
-  const int W = blockDim.x >> 5;
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(sm);      // [n_buckets]
   const int q = blockIdx.x % Q;
   const int64_t seg = blockIdx.x / Q;
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  zero_counters(cnt, W * n_buckets);
+  for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) cnt[b] = 0u;
   __syncthreads();
-  warp_count(bucket + seg * L, (int64_t)q * P + (int64_t)w * PW, PW, L, lane,
-             cnt + w * n_buckets, n_buckets, status);
+  const int32_t* sb = bucket + seg * L;
+  const int64_t p0 = (int64_t)q * P;
+  for (int i = threadIdx.x; i < P; i += blockDim.x) {
+    const uint32_t b = load_bucket(sb, p0 + i, L, n_buckets, status);
+    if (b != 0xffffffffu) atomicAdd(&cnt[b], 1u);
+  }
   __syncthreads();
   int32_t* out = counts + (seg * Q + q) * (int64_t)n_buckets;
-  for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
-    int tot = 0;
-    for (int ww = 0; ww < W; ++ww) tot += cnt[ww * n_buckets + b];
-    out[b] = tot;
-  }
+  for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) out[b] = (int32_t)cnt[b];
 }
 
-// Exclusive scan of v[0, n) in place by the whole block (n <= blockDim * 32
-// per thread run); `red` holds 64 ints of scratch.
+// Exclusive scan of v[0, n) in place by the whole block; `red` holds 64 ints
+// of scratch.
 __device__ __forceinline__ void block_exclusive_scan(int32_t* v, int n, int* red) {
   const int T = blockDim.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
   const int per = (n + T - 1) / T;
@@ -309,7 +339,10 @@ sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restric
   const int q = blockIdx.x % Q;
   const int64_t seg = blockIdx.x / Q;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  zero_counters(cnt, W * n_buckets);
+  {
+    uint32_t* c32 = reinterpret_cast<uint32_t*>(cnt);   // W * n_buckets is even
+    for (int i = threadIdx.x; i < W * n_buckets / 2; i += blockDim.x) c32[i] = 0u;
+  }
   // totals of the segment per bucket, and the counts of the blocks before q
   const int32_t* cs = counts + seg * Q * (int64_t)n_buckets;
   for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
@@ -325,9 +358,16 @@ sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restric
   __syncthreads();
   block_exclusive_scan(base, n_buckets, red);
   for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) base[b] += pre[b];
-  const int32_t* sb = bucket + seg * L;
+  const int32_t* sbk = bucket + seg * L;
   const int64_t i0 = (int64_t)q * P + (int64_t)w * PW;
-  warp_count(sb, i0, PW, L, lane, cnt + w * n_buckets, n_buckets, nullptr);
+  uint16_t* mine = cnt + w * n_buckets;
+  // pass 1: this warp's count of every bucket
+  for (int st = 0; st < PW; st += 32) {
+    const uint32_t b = load_bucket(sbk, i0 + st + lane, L, n_buckets, nullptr);
+    const StepRank r = rank_step(b, lane);
+    if (r.live && r.last) mine[r.bucket] = (uint16_t)(mine[r.bucket] + r.len);
+    __syncwarp();
+  }
   __syncthreads();
   // exclusive prefix over warps: cnt[w][b] becomes the start of warp w's run
   for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
@@ -339,20 +379,14 @@ sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restric
     }
   }
   __syncthreads();
-  uint16_t* mine = cnt + w * n_buckets;
+  // pass 2: every position to base + warp run + earlier steps + rank
   int32_t* out = perm + seg * L;
   for (int st = 0; st < PW; st += 32) {
-    const int64_t i = i0 + st + lane;
-    uint32_t b = 0xffffffffu;
-    if (i < L) {
-      b = (uint32_t)__ldg(sb + i);
-      if (b >= (uint32_t)n_buckets) b = (uint32_t)n_buckets - 1;
-    }
-    const uint32_t peers = __match_any_sync(0xffffffffu, b);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    if (i < L) out[base[b] + mine[b] + rank] = (int32_t)i;
+    const uint32_t b = load_bucket(sbk, i0 + st + lane, L, n_buckets, nullptr);
+    const StepRank r = rank_step(b, lane);
+    if (r.live) out[base[r.bucket] + mine[r.bucket] + r.rank] = (int32_t)(i0 + st + r.src);
     __syncwarp();
-    if (i < L && lane == __ffs(peers) - 1) mine[b] = (uint16_t)(mine[b] + __popc(peers));
+    if (r.live && r.last) mine[r.bucket] = (uint16_t)(mine[r.bucket] + r.len);
     __syncwarp();
   }
 }
@@ -396,7 +430,7 @@ cudaError_t launch_sort(const lsh_problem& p, const int32_t* bucket, int32_t* pe
   const int64_t rows = S * p.n_buckets;
   if (warp_path(p)) {
     const WarpGeo g = warp_geo(p);
-    const size_t sm_count_k = (size_t)g.W * p.n_buckets * 2;
+    const size_t sm_count_k = (size_t)p.n_buckets * 4;
     cudaError_t e = cudaFuncSetAttribute(sort_count_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_count_k);
     if (e != cudaSuccess) return e;
@@ -404,8 +438,8 @@ cudaError_t launch_sort(const lsh_problem& p, const int32_t* bucket, int32_t* pe
                              (int)g.smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)(S * g.Q);
-    sort_count_kernel<<<grid, g.W * 32, sm_count_k, s>>>(bucket, ws.counts, p.L, p.n_buckets,
-                                                         g.PW, g.P, g.Q, status);
+    sort_count_kernel<<<grid, 1024, sm_count_k, s>>>(bucket, ws.counts, p.L, p.n_buckets, g.P,
+                                                     g.Q, status);
     sort_scatter_kernel<<<grid, g.W * 32, g.smem, s>>>(bucket, ws.counts, perm, p.L, p.n_buckets,
                                                        g.PW, g.P, g.Q);
     note_launch(2);
