@@ -10,11 +10,11 @@
 //    blocks of 8K-32K consecutive positions, one CTA each (see the counting
 //    path below): block totals per bucket from shared-memory atomics, then a
 //    scatter kernel that forms the bucket bases itself and ranks positions
-//    with warp-level bitonic sorts of (bucket, lane) keys;
+//    within each warp step by ballots over the bucket bits;
 //  * larger bucket counts: per 4096-position tile the packed keys
 //    (bucket << 12 | local index) are sorted in shared memory by a bitonic
 //    network; row_scan / bucket_scan form the bases; scatter places them.
-// Ranks follow position order inside a warp step (the lane breaks ties),
+// Ranks follow position order inside a warp step (lane order),
 // across the steps of a warp (in order), across the warps of a block
 // (exclusive prefix of their counts) and across blocks (counts of the blocks
 // before), so the whole sort is stable.
@@ -187,12 +187,12 @@ scatter_kernel(const uint32_t* __restrict__ sorted, const int32_t* __restrict__ 
 //   sort_scatter_kernel: bucket bases of the segment (exclusive scan of the
 //                        totals over buckets) plus the counts of the blocks
 //                        before q; then each warp takes its positions 32 at a
-//                        time, sorts the 32 (bucket, lane) keys with a warp
-//                        bitonic network so equal buckets form contiguous
-//                        segments in lane order, and ranks each position
-//                        within its segment. A first pass counts per warp, an
-//                        exclusive prefix over warps gives each warp's run, and
-//                        a second pass places every position at its slot.
+//                        time and finds, with one ballot per bucket bit, the
+//                        lanes that share each lane's bucket: a position's rank
+//                        is the number of such lanes below it. A first pass
+//                        counts per warp, an exclusive prefix over warps gives
+//                        each warp's run, and a second pass places every
+//                        position at its slot.
 constexpr int kWarpMaxBuckets = 8192;
 constexpr int kSortSmemBudget = 200 * 1024;
 
@@ -201,15 +201,26 @@ struct WarpGeo {
   int PW;       // positions per warp (multiple of 32)
   int P;        // positions per CTA = W * PW
   int Q;        // CTAs per segment
+  bool scanned; // block prefixes and bucket bases from the two scan kernels
   size_t smem;  // dynamic shared memory of the scatter kernel (the larger)
 };
+
+constexpr int64_t kDirectCounts = 65536;   // Q * n_buckets read by each scatter CTA at most
 
 WarpGeo warp_geo(const lsh_problem& p) {
   WarpGeo g;
   const int nb = p.n_buckets;
+  const int64_t S = (int64_t)p.B * p.H * p.n_rounds;
   g.W = (int)std::min<int64_t>(32, (kSortSmemBudget - 8 * (int64_t)nb) / (2 * (int64_t)nb));
   // a few blocks per segment (at most ~16) of 8K..32K positions
   int64_t P = std::min<int64_t>(32768, std::max<int64_t>(8192, ((int64_t)p.L + 15) / 16));
+  int64_t Q = ((int64_t)p.L + P - 1) / P;
+  g.scanned = Q * nb > kDirectCounts || S * Q < 148;
+  if (g.scanned) {
+    // smaller blocks, about two CTAs per SM over all segments; the scan
+    // kernels then give each CTA its bases
+    P = std::min<int64_t>(32768, std::max<int64_t>(32 * g.W, S * p.L / 296));
+  }
   g.PW = (int)((P + 32 * g.W - 1) / (32 * g.W)) * 32;
   g.P = g.W * g.PW;
   g.Q = (int)(((int64_t)p.L + g.P - 1) / g.P);
@@ -230,44 +241,18 @@ __device__ __forceinline__ uint32_t load_bucket(const int32_t* __restrict__ seg_
   return b;
 }
 
-// Sorts the warp's 32 keys ascending (bitonic network over lanes).
-__device__ __forceinline__ uint32_t warp_sort32(uint32_t key, int lane) {
-#pragma unroll
-  for (int k = 2; k <= 32; k <<= 1) {
-#pragma unroll
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      const uint32_t o = __shfl_xor_sync(0xffffffffu, key, j);
-      const bool up = (lane & k) == 0, lower = (lane & j) == 0;
-      key = (lower == up) ? min(key, o) : max(key, o);
-    }
+// The lanes of the warp whose bucket equals this lane's: one ballot per bucket
+// bit (nbits of them), each lane keeping the lanes that agree on the bit.
+// Lanes past the end of the segment (bucket 0xffffffff) are excluded.
+__device__ __forceinline__ uint32_t same_bucket_lanes(uint32_t b, int nbits) {
+  const bool live = b != 0xffffffffu;
+  uint32_t eq = __ballot_sync(0xffffffffu, live);
+  for (int k = 0; k < nbits; ++k) {
+    const bool bit = (b >> k) & 1u;
+    const uint32_t m = __ballot_sync(0xffffffffu, bit);
+    eq &= bit ? m : ~m;
   }
-  return key;
-}
-
-// One step of 32 positions: after sorting (bucket << 5 | lane) keys, lane k
-// holds sorted entry k: its bucket, the lane (position offset) it came from,
-// its rank among the entries of its bucket, and whether it ends the bucket's
-// segment (then `len` is the segment's length).
-struct StepRank {
-  uint32_t bucket;
-  int src, rank, len;
-  bool live, last;
-};
-__device__ __forceinline__ StepRank rank_step(uint32_t b, int lane) {
-  const uint32_t key = warp_sort32(b == 0xffffffffu ? 0xffffffffu : (b << 5) | (uint32_t)lane, lane);
-  StepRank r;
-  r.live = key != 0xffffffffu;
-  r.bucket = key >> 5;
-  r.src = (int)(key & 31u);
-  const uint32_t prev = __shfl_up_sync(0xffffffffu, r.bucket, 1);
-  const uint32_t next = __shfl_down_sync(0xffffffffu, r.bucket, 1);
-  const bool first = lane == 0 || prev != r.bucket;
-  r.last = lane == 31 || next != r.bucket;
-  const uint32_t starts = __ballot_sync(0xffffffffu, first);
-  const int seg0 = 31 - __clz(starts & (0xffffffffu >> (31 - lane)));
-  r.rank = lane - seg0;
-  r.len = r.rank + 1;
-  return r;
+  return eq;
 }
 
 __global__ void __launch_bounds__(1024)
@@ -327,9 +312,36 @@ __device__ __forceinline__ void block_exclusive_scan(int32_t* v, int n, int* red
   __syncthreads();
 }
 
+// For every (segment, bucket): exclusive prefix of the block counts over the
+// blocks, in place, and the bucket's total.
+__global__ void __launch_bounds__(256)
+sort_qscan_kernel(int32_t* __restrict__ counts, int32_t* __restrict__ totals, int n_buckets, int Q,
+                  int64_t rows) {
+  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // seg * n_buckets + b
+  if (k >= rows) return;
+  const int64_t seg = k / n_buckets, b = k - seg * n_buckets;
+  int32_t* c = counts + seg * Q * (int64_t)n_buckets + b;
+  int run = 0;
+  for (int q = 0; q < Q; ++q) {
+    const int v = c[(int64_t)q * n_buckets];
+    c[(int64_t)q * n_buckets] = run;
+    run += v;
+  }
+  totals[k] = run;
+}
+
+// For every segment: exclusive scan of the bucket totals, in place (the
+// bucket bases).
+__global__ void __launch_bounds__(1024)
+sort_bscan_kernel(int32_t* __restrict__ totals, int n_buckets) {
+  __shared__ int red[64];
+  block_exclusive_scan(totals + (int64_t)blockIdx.x * n_buckets, n_buckets, red);
+}
+
 __global__ void __launch_bounds__(1024)
 sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restrict__ counts,
-                    int32_t* __restrict__ perm, int L, int n_buckets, int PW, int P, int Q) {
+                    const int32_t* __restrict__ bases, int32_t* __restrict__ perm, int L,
+                    int n_buckets, int PW, int P, int Q) {
   extern __shared__ __align__(16) uint8_t sm[];
   const int W = blockDim.x >> 5;
   uint16_t* cnt = reinterpret_cast<uint16_t*>(sm);                                // [W][nb]
@@ -343,29 +355,40 @@ sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restric
     uint32_t* c32 = reinterpret_cast<uint32_t*>(cnt);   // W * n_buckets is even
     for (int i = threadIdx.x; i < W * n_buckets / 2; i += blockDim.x) c32[i] = 0u;
   }
-  // totals of the segment per bucket, and the counts of the blocks before q
   const int32_t* cs = counts + seg * Q * (int64_t)n_buckets;
-  for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
-    int tot = 0, before = 0;
-    for (int qq = 0; qq < Q; ++qq) {
-      const int c = __ldg(cs + (int64_t)qq * n_buckets + b);
-      tot += c;
-      if (qq < q) before += c;
+  if (bases) {
+    // from the scan kernels: bucket bases, and the counts before this block
+    const int32_t* bs = bases + seg * (int64_t)n_buckets;
+    for (int b = threadIdx.x; b < n_buckets; b += blockDim.x)
+      base[b] = __ldg(bs + b) + __ldg(cs + (int64_t)q * n_buckets + b);
+    __syncthreads();
+  } else {
+    // totals of the segment per bucket, and the counts of the blocks before q
+    for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
+      int tot = 0, before = 0;
+      for (int qq = 0; qq < Q; ++qq) {
+        const int c = __ldg(cs + (int64_t)qq * n_buckets + b);
+        tot += c;
+        if (qq < q) before += c;
+      }
+      base[b] = tot;
+      pre[b] = before;
     }
-    base[b] = tot;
-    pre[b] = before;
+    __syncthreads();
+    block_exclusive_scan(base, n_buckets, red);
+    for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) base[b] += pre[b];
   }
-  __syncthreads();
-  block_exclusive_scan(base, n_buckets, red);
-  for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) base[b] += pre[b];
   const int32_t* sbk = bucket + seg * L;
   const int64_t i0 = (int64_t)q * P + (int64_t)w * PW;
   uint16_t* mine = cnt + w * n_buckets;
-  // pass 1: this warp's count of every bucket
+  const int nbits = 32 - __clz(n_buckets - 1);
+  const uint32_t below = (1u << lane) - 1u;
+  // pass 1: this warp's count of every bucket (the lowest lane of each group
+  // of equal buckets adds the group's size)
   for (int st = 0; st < PW; st += 32) {
     const uint32_t b = load_bucket(sbk, i0 + st + lane, L, n_buckets, nullptr);
-    const StepRank r = rank_step(b, lane);
-    if (r.live && r.last) mine[r.bucket] = (uint16_t)(mine[r.bucket] + r.len);
+    const uint32_t eq = same_bucket_lanes(b, nbits);
+    if (b != 0xffffffffu && (eq & below) == 0u) mine[b] = (uint16_t)(mine[b] + __popc(eq));
     __syncwarp();
   }
   __syncthreads();
@@ -383,10 +406,10 @@ sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restric
   int32_t* out = perm + seg * L;
   for (int st = 0; st < PW; st += 32) {
     const uint32_t b = load_bucket(sbk, i0 + st + lane, L, n_buckets, nullptr);
-    const StepRank r = rank_step(b, lane);
-    if (r.live) out[base[r.bucket] + mine[r.bucket] + r.rank] = (int32_t)(i0 + st + r.src);
+    const uint32_t eq = same_bucket_lanes(b, nbits);
+    if (b != 0xffffffffu) out[base[b] + mine[b] + __popc(eq & below)] = (int32_t)(i0 + st + lane);
     __syncwarp();
-    if (r.live && r.last) mine[r.bucket] = (uint16_t)(mine[r.bucket] + r.len);
+    if (b != 0xffffffffu && (eq & below) == 0u) mine[b] = (uint16_t)(mine[b] + __popc(eq));
     __syncwarp();
   }
 }
@@ -397,7 +420,9 @@ bool warp_path(const lsh_problem& p) { return p.n_buckets <= kWarpMaxBuckets; }
 
 size_t sort_ws_bytes(const lsh_problem& p) {
   const int64_t S = (int64_t)p.B * p.H * p.n_rounds;
-  if (warp_path(p)) return align_up((size_t)S * warp_geo(p).Q * p.n_buckets * 4, 256);
+  if (warp_path(p))
+    return align_up((size_t)S * warp_geo(p).Q * p.n_buckets * 4, 256) +
+           align_up((size_t)S * p.n_buckets * 4, 256);
   const int64_t tiles = (p.L + kTile - 1) / kTile;
   size_t b = align_up((size_t)S * p.L * 4, 256);
   b += align_up((size_t)S * p.n_buckets * tiles * 4, 256);
@@ -412,7 +437,7 @@ SortWs sort_ws_carve(const lsh_problem& p, void* ws) {
   if (warp_path(p)) {
     w.sorted = nullptr;
     w.counts = (int32_t*)c;
-    w.base = nullptr;
+    w.base = (int32_t*)(c + align_up((size_t)S * warp_geo(p).Q * p.n_buckets * 4, 256));
     return w;
   }
   const int64_t tiles = (p.L + kTile - 1) / kTile;
@@ -440,9 +465,15 @@ cudaError_t launch_sort(const lsh_problem& p, const int32_t* bucket, int32_t* pe
     const unsigned grid = (unsigned)(S * g.Q);
     sort_count_kernel<<<grid, 1024, sm_count_k, s>>>(bucket, ws.counts, p.L, p.n_buckets, g.P,
                                                      g.Q, status);
-    sort_scatter_kernel<<<grid, g.W * 32, g.smem, s>>>(bucket, ws.counts, perm, p.L, p.n_buckets,
-                                                       g.PW, g.P, g.Q);
-    note_launch(2);
+    if (g.scanned) {
+      sort_qscan_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(ws.counts, ws.base,
+                                                                       p.n_buckets, g.Q, rows);
+      sort_bscan_kernel<<<(unsigned)S, 1024, 0, s>>>(ws.base, p.n_buckets);
+    }
+    sort_scatter_kernel<<<grid, g.W * 32, g.smem, s>>>(bucket, ws.counts,
+                                                       g.scanned ? ws.base : nullptr, perm, p.L,
+                                                       p.n_buckets, g.PW, g.P, g.Q);
+    note_launch(g.scanned ? 4 : 2);
     return cudaGetLastError();
   }
   const int tiles = (p.L + kTile - 1) / kTile;
