@@ -27,11 +27,14 @@
 //        so that the next item of the same unit adds its own terms on top.
 //        At the end of a unit it is stored on its own (the edge rows below).
 // The finished rows dV and scale*dK of an item are stored, converted to fp16,
-// as per-round partial gradients in sorted (slot) order — 128 consecutive
-// rows, two TMA tile stores per tensor; unit-end R1 rows go to a small edge
-// buffer. A second kernel then sums, for every token, its rows of all rounds
-// (located through the inverse permutation) into dqk and dv, so no atomics
-// are needed anywhere.
+// as per-round partial gradients in token order: each flush thread writes its
+// key row's two 128-byte rows at the row's position, so every round's
+// partial is a plain (position, 64) array. Unit-end R1 rows go to a small
+// edge buffer, and the first item of the next unit records, per position of
+// its first chunk, which edge row belongs to it (-1 for every other
+// position). A second kernel then streams the rounds' partials of every
+// token, adds its edge rows and writes dqk and dv, so no atomics and no
+// inverse permutation are needed.
 //
 // TMEM (512 columns): two S^T|dP^T buffers (steps alternate) and two
 // dV|dK accumulator sets (items alternate), so that the S^T/dP^T products
@@ -42,9 +45,11 @@
 //   warps 0-2  : producers — cp.async gathers of the fp16 copies of x, dout
 //                (3 chunks) and v (2 chunks) into a 2-slot ring, per-query
 //                position, log2-scaled LSE and D;
-//   warp 3     : TMEM allocation and the MMA-issuing thread;
-//   warps 4-7  : gradient flush of the previous item (one thread per row,
-//                fp16 staging in shared memory, TMA stores);
+//   warp 3     : TMEM allocation and the MMA issue (the warp waits
+//                converged; one elected lane issues each MMA and commit);
+//   warps 4-7  : gradient flush of the previous item (one thread per key
+//                row: TMEM -> fp16 -> a padded staging row -> one bulk copy
+//                to the row's place in the partial arrays);
 //   warps 8-23 : four softmax warpgroups, two per S^T buffer (even and odd
 //                steps), one thread per key row and 32 of the block's 64
 //                query columns each.
@@ -70,7 +75,8 @@ constexpr int kX = 0, kV = 3 * kTile, kDo = 5 * kTile;
 constexpr int kSlotBytes = 8 * kTile;  // 64 KB
 constexpr int kDsBlock = 128 * 128;    // 128 key rows x 64 query columns
 constexpr int kDsBytes = 4 * kDsBlock; // dS^T blocks 0,1,2 + a zero block
-constexpr int kStageBytes = 128 * 128; // 128 fp16 rows, 128-byte swizzle
+constexpr int kStageRow = 144;         // fp16 row of 128 bytes + 16 bytes of padding
+constexpr int kStageBytes = 128 * kStageRow;
 constexpr int kThreads = 768;
 constexpr int kProducers = 96;
 // Launched at 80 registers per thread (768 threads); producers/MMA and flush
@@ -151,9 +157,13 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 // one lane never leaves the others inside a warp-collective instruction.
 __device__ __forceinline__ bool warp_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
 
-// Converts 64 fp32 TMEM columns of this thread's lane, times `sc`, to fp16
-// and writes them as row `row` of a 128-byte-swizzled staging tile.
-__device__ __forceinline__ void stage_row(uint32_t ta, float sc, uint8_t* stage, int row) {
+// Converts 64 fp32 TMEM columns of this thread's lane, times `sc`, to fp16,
+// places them in this thread's row of the staging area (rows 144 bytes apart,
+// so the 16-byte stores of eight consecutive rows fall in different banks)
+// and copies the 128 bytes to the global row `dst` with one bulk copy. The
+// staging row is free again when the function returns.
+__device__ __forceinline__ void put_row(uint32_t ta, float sc, uint8_t* srow, __half* dst,
+                                        bool live) {
 #pragma unroll
   for (int h = 0; h < 4; ++h) {
     uint32_t a[16];
@@ -163,13 +173,14 @@ __device__ __forceinline__ void stage_row(uint32_t ta, float sc, uint8_t* stage,
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       pk[i] = pack_f16x2(__uint_as_float(a[2 * i]) * sc, __uint_as_float(a[2 * i + 1]) * sc);
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int ch = h * 2 + c;
-      *reinterpret_cast<uint4*>(stage + row * 128 + ((ch ^ (row & 7)) << 4)) =
-          make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-    }
+    uint4* d = reinterpret_cast<uint4*>(srow) + 2 * h;
+    d[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    d[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
   }
+  fence_proxy_async();
+  if (live) bulk_store(dst, smem_u32(srow), 128);
+  bulk_commit();
+  bulk_wait_read_all();
 }
 
 // ---- MMA issue helpers (one thread). Descriptor lower words: `sl` is the
@@ -217,7 +228,7 @@ __device__ __forceinline__ void bwd_issue_r(uint32_t d, uint32_t ds, uint32_t sl
     mma_ss_w(d, ds + 128 * ks, xk + 128 * ks, kDescHi1024, kIdNN, acc || ks > KS0);
 }
 __device__ __forceinline__ bool bwd_wait_p(BwdBar* bar, int g, volatile int* abort, int* status) {
-  return mbar_wait(&bar->p_full[g & 1], (uint32_t)(g >> 1) & 1u, abort, status);
+  return __all_sync(0xffffffffu, mbar_wait(&bar->p_full[g & 1], (uint32_t)(g >> 1) & 1u, abort, status));
 }
 
 template <bool kCausal>
@@ -225,17 +236,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __half* __restrict__ qk, const __half* __restrict__ v,
                    const __half* __restrict__ dout, const int32_t* __restrict__ perm,
                    const float* __restrict__ lse, const float* __restrict__ Dg,
-                   const __grid_constant__ CUtensorMap map_dv,
-                   const __grid_constant__ CUtensorMap map_dqk,
-                   const __grid_constant__ CUtensorMap map_edge, int L, int n_rounds,
+                   __half* __restrict__ part_dv, __half* __restrict__ part_dqk,
+                   __half* __restrict__ edge, int32_t* __restrict__ emap, int L, int n_rounds,
                    float scale, float scale_log2, int n_units, int units_per_seg,
                    int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* slots = smem;
   uint8_t* dsb = slots + kSlots * kSlotBytes;
-  uint8_t* stage_base = dsb + kDsBytes;
-  BwdBar* bar = (BwdBar*)(stage_base + kStageBytes);
+  uint8_t* stage = dsb + kDsBytes;
+  BwdBar* bar = (BwdBar*)(stage + kStageBytes);
   volatile int* abort = &bar->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -354,8 +364,9 @@ attn_bwd_tc_kernel(const __half* __restrict__ qk, const __half* __restrict__ v,
         have = have_next;
         ++n;
       }
-    } else if (lane == 0) {
-      // ---------------------------------------------- MMA issuer
+    } else {
+      // ---------------------------------------------- MMA issuer (whole warp
+      // converged; each MMA / commit issued by one elected lane)
       JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
       Job cur, nxt;
       bool have = it.next(cur);
@@ -364,7 +375,7 @@ attn_bwd_tc_kernel(const __half* __restrict__ qk, const __half* __restrict__ v,
       const uint32_t ds_lo = (smem_u32(dsb) >> 4) | desc_lbo(kDsBlock);
       int seen0 = 0, seen1 = 0;   // acc_free completions waited for, per set
       if (have) {
-        ok = mbar_wait(&bar->slot_full[0], 0u, abort, status);
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar->slot_full[0], 0u, abort, status));
         if (ok) {
           tc_fence_after();
           const int nc = min(3, n_chunks - 2 * cur.p);
@@ -388,12 +399,13 @@ attn_bwd_tc_kernel(const __half* __restrict__ qk, const __half* __restrict__ v,
         {
           const int need = n >> 1;
           int& seen = a ? seen1 : seen0;
-          while (ok && seen < need) ok = mbar_wait(&bar->acc_free[a], (uint32_t)(seen++) & 1u, abort, status);
+          while (ok && seen < need)
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar->acc_free[a], (uint32_t)(seen++) & 1u, abort, status));
           if (prev_r1_alone) {
             const int b = a ^ 1, need_b = ((n - 1) >> 1) + 1;
             int& seen_b = b ? seen1 : seen0;
             while (ok && seen_b < need_b)
-              ok = mbar_wait(&bar->acc_free[b], (uint32_t)(seen_b++) & 1u, abort, status);
+              ok = __all_sync(0xffffffffu, mbar_wait(&bar->acc_free[b], (uint32_t)(seen_b++) & 1u, abort, status));
           }
           if (!ok) break;
         }
@@ -410,7 +422,7 @@ attn_bwd_tc_kernel(const __half* __restrict__ qk, const __half* __restrict__ v,
         uint32_t sl_next = 0;
         if (have_next) {
           const int sn = (n + 1) % kSlots;
-          if (!mbar_wait(&bar->slot_full[sn], (uint32_t)((n + 1) / kSlots) & 1u, abort, status))
+          if (!__all_sync(0xffffffffu, mbar_wait(&bar->slot_full[sn], (uint32_t)((n + 1) / kSlots) & 1u, abort, status)))
             break;
           tc_fence_after();
           nc_next = min(3, n_chunks - 2 * nxt.p);
@@ -425,7 +437,7 @@ attn_bwd_tc_kernel(const __half* __restrict__ qk, const __half* __restrict__ v,
           const int b = a ^ 1, need_b = (n + 1) >> 1;
           int& seen_b = b ? seen1 : seen0;
           while (ok && seen_b < need_b)
-            ok = mbar_wait(&bar->acc_free[b], (uint32_t)(seen_b++) & 1u, abort, status);
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar->acc_free[b], (uint32_t)(seen_b++) & 1u, abort, status));
           if (!ok) break;
           tc_fence_after();
           // block 2's queries see only the keys of chunk 2p+1 (rows 64-127;
@@ -452,50 +464,34 @@ attn_bwd_tc_kernel(const __half* __restrict__ qk, const __half* __restrict__ v,
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
-    const bool issuer = threadIdx.x == 128;
+    uint8_t* srow = stage + row * kStageRow;
     JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
     Job j;
     int n = 0;
-    // stage -> TMA store of rows [0, 64 nh) to (0, y) of `map`
-    auto store_rows = [&](const CUtensorMap* map, int y, int nh) {
-      fence_proxy_async();
-      named_sync(2, 128);
-      if (issuer) {
-        tma_store_2d(map, 0, y, stage_base);
-        if (nh > 1) tma_store_2d(map, 0, y + 64, stage_base + 64 * 128);
-        bulk_commit();
-        bulk_wait_read_all();
-      }
-      named_sync(2, 128);
-    };
     while (it.next(j)) {
       const int a = n & 1;
-      const bool got = mbar_wait(&bar->g_full[a], (uint32_t)(n >> 1) & 1u, abort, status);
-      if (!group_ok(2, 128, got)) break;
+      if (!warp_ok(mbar_wait(&bar->g_full[a], (uint32_t)(n >> 1) & 1u, abort, status))) break;
       tc_fence_after();
       const int nc = min(3, n_chunks - 2 * j.p);
-      const int nh = min(nc, 2);                 // 64-row halves of key rows present
-      const int y = (int)(j.seg * L) + 2 * j.p * kM;
+      const bool live = row < 64 * min(nc, 2);   // key rows present
+      const int tp = bar->tok[n & 3][row];        // this key row's position
+      const int64_t rr = j.seg * L + (live ? tp : 0);
       const uint32_t acc = tl + kColAcc + (uint32_t)a * 128;
       const bool r1 = j.last && nc == 3;
-      stage_row(acc, 1.f, stage_base, row);
-      store_rows(&map_dv, y, nh);
-      stage_row(acc + 64, scale, stage_base, row);
-      if (!r1) {
-        tc_fence_before();
-        mbar_arrive(&bar->acc_free[a]);
-      }
-      store_rows(&map_dqk, y, nh);
-      if (r1) {
-        // R1 rows (chunk 2p+2) that no later item of this unit picks up
-        if (q < 2) stage_row(tl + kColAcc + (uint32_t)(a ^ 1) * 128 + 64, scale, stage_base, row);
-        tc_fence_before();
-        mbar_arrive(&bar->acc_free[a]);
-        store_rows(&map_edge, (int)(j.seg * units_per_seg + j.p / kUnit) * kM, 1);
-      }
+      const int unit = (int)(j.seg * units_per_seg + j.p / kUnit);
+      put_row(acc, 1.f, srow, part_dv + rr * 64, live);
+      put_row(acc + 64, scale, srow, part_dqk + rr * 64, live);
+      // the rows of a unit's first chunk (after the first unit) take the R1
+      // rows that the previous unit's last item stored on its own
+      if (live) emap[rr] = (j.first && j.p > 0 && row < kM) ? (unit - 1) * kM + row : -1;
+      if (r1 && q < 2)
+        put_row(tl + kColAcc + (uint32_t)(a ^ 1) * 128 + 64, scale, srow,
+                edge + ((int64_t)unit * kM + row) * 64, true);
+      tc_fence_before();
+      mbar_arrive(&bar->acc_free[a]);
       ++n;
     }
-    if (issuer) bulk_wait_all();
+    bulk_wait_all();
   } else {
     // ------------------------------------------------ softmax: P^T and dS^T
     // Two warpgroups per S^T buffer, each owning 32 of the block's 64 query
@@ -650,22 +646,6 @@ bwd_prep_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
                                                     bf16x2_to_f16x2(g.z), bf16x2_to_f16x2(g.w));
 }
 
-// inv[seg][perm[seg][i]] = i: the slot of every position in every round.
-__global__ void __launch_bounds__(256)
-inverse_perm_kernel(const int32_t* __restrict__ perm, int32_t* __restrict__ inv, int L,
-                    int64_t total, int* status) {
-  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (k >= total) return;
-  const int64_t seg = k / L;
-  const int i = (int)(k - seg * L);
-  const int pos = perm[k];
-  if ((unsigned)pos >= (unsigned)L) {
-    record_status(status, (int)LSH_ERR_DEVICE_CHECK);
-    return;
-  }
-  inv[seg * L + pos] = i;
-}
-
 __device__ __forceinline__ void add8_f16(float (&acc)[8], const uint4 w) {
   const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -676,18 +656,17 @@ __device__ __forceinline__ void add8_f16(float (&acc)[8], const uint4 w) {
   }
 }
 
-// dv, dqk of every token: the sum over rounds of its partial rows (slot
-// inv[seg][pos] of segment seg = bh * n_rounds + r), plus the unit-end R1
-// row where its slot opens a unit; dv also takes dout for a token that
-// attended only to itself (final LSE of -inf). Eight threads per token;
-// the slots of two rounds are looked up first and their four rows loaded
-// together, to keep more reads in flight.
+// dv, dqk of every token: the sum over rounds of its partial rows (row pos
+// of segment bh * n_rounds + r), plus the R1 row that emap names where the
+// token opens a unit; dv also takes dout for a token that attended only to
+// itself (final LSE of -inf). Eight threads per token; the rows of two
+// rounds are loaded together, to keep more reads in flight.
 __global__ void __launch_bounds__(256)
-unsort_kernel(const __half* __restrict__ part_dv, const __half* __restrict__ part_dqk,
-              const __half* __restrict__ edge, const int32_t* __restrict__ inv,
-              const float* __restrict__ lse, const __nv_bfloat16* __restrict__ dout,
-              float* __restrict__ dqk, float* __restrict__ dv, int L, int n_rounds,
-              int units_per_seg, int64_t N, int* status) {
+sum_rounds_kernel(const __half* __restrict__ part_dv, const __half* __restrict__ part_dqk,
+                  const __half* __restrict__ edge, const int32_t* __restrict__ emap,
+                  const float* __restrict__ lse, const __nv_bfloat16* __restrict__ dout,
+                  float* __restrict__ dqk, float* __restrict__ dv, int L, int n_rounds,
+                  int64_t n_edge_rows, int64_t N, int* status) {
   const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
   const int c8 = (threadIdx.x & 7) * 8;
   if (t >= N) return;
@@ -698,29 +677,25 @@ unsort_kernel(const __half* __restrict__ part_dv, const __half* __restrict__ par
   for (int e = 0; e < 8; ++e) a[e] = b[e] = 0.f;
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
   for (int r0 = 0; r0 < n_rounds; r0 += 2) {
-    int slot[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k)
-      slot[k] = r0 + k < n_rounds ? __ldg(inv + (bh * n_rounds + r0 + k) * L + pos) : 0;
     uint4 ua[2], ub[2];
+    int er[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const bool live = r0 + k < n_rounds;
-      const bool ok = (unsigned)slot[k] < (unsigned)L;
-      if (live && !ok) record_status(status, (int)LSH_ERR_DEVICE_CHECK);
-      const int64_t row = (bh * n_rounds + r0 + k) * L + (ok ? slot[k] : 0);
-      ua[k] = live && ok ? __ldg(reinterpret_cast<const uint4*>(part_dv + row * 64 + c8)) : zero;
-      ub[k] = live && ok ? __ldg(reinterpret_cast<const uint4*>(part_dqk + row * 64 + c8)) : zero;
+      const int64_t row = (bh * n_rounds + (live ? r0 + k : 0)) * L + pos;
+      ua[k] = live ? __ldg(reinterpret_cast<const uint4*>(part_dv + row * 64 + c8)) : zero;
+      ub[k] = live ? __ldg(reinterpret_cast<const uint4*>(part_dqk + row * 64 + c8)) : zero;
+      er[k] = live ? __ldg(emap + row) : -1;
     }
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       add8_f16(a, ua[k]);
       add8_f16(b, ub[k]);
-      const int i = slot[k], c = i / kM;
-      if (r0 + k < n_rounds && (unsigned)i < (unsigned)L && c > 0 && c % (2 * kUnit) == 0) {
-        const int64_t er = ((bh * n_rounds + r0 + k) * units_per_seg + c / (2 * kUnit) - 1) * kM +
-                           (i % kM);
-        add8_f16(b, __ldg(reinterpret_cast<const uint4*>(edge + er * 64 + c8)));
+      if (er[k] >= 0) {
+        if (er[k] < n_edge_rows)
+          add8_f16(b, __ldg(reinterpret_cast<const uint4*>(edge + (int64_t)er[k] * 64 + c8)));
+        else
+          record_status(status, (int)LSH_ERR_DEVICE_CHECK);
       }
     }
   }
@@ -759,7 +734,7 @@ struct TcWs {
   __half* x16;
   __half* v16;
   __half* g16;
-  int32_t* inv;
+  int32_t* emap;
   __half* part_dv;
   __half* part_dqk;
   __half* edge;
@@ -781,7 +756,7 @@ TcWs tc_ws(const lsh_problem& p, void* base) {
   off += al(toks * 64 * 2);
   w.g16 = (__half*)(c + off);
   off += al(toks * 64 * 2);
-  w.inv = (int32_t*)(c + off);
+  w.emap = (int32_t*)(c + off);
   off += al(rows * 4);
   w.part_dv = (__half*)(c + off);
   off += al(rows * 64 * 2);
@@ -810,20 +785,10 @@ cudaError_t launch_attn_bwd_tc(const lsh_problem& p, const void* qk, const void*
   const int units_per_seg = (n_pairs + kUnit - 1) / kUnit;
   const int64_t n_segs = (int64_t)p.B * p.H * p.n_rounds;
   const int64_t n_units = n_segs * units_per_seg;
-  const int64_t rows = n_segs * p.L;
   const int64_t N = (int64_t)p.B * p.H * p.L;
-  // per-round partial gradients (fp16 rows in slot order) and unit-end R1 rows,
-  // written by 64-row TMA boxes with 128-byte swizzle
-  CUtensorMap m_dv, m_dqk, m_edge;
-  if (!encode_tmap_2d_16bit(&m_dv, w.part_dv, 64, (uint64_t)rows, 128, 64, 64) ||
-      !encode_tmap_2d_16bit(&m_dqk, w.part_dqk, 64, (uint64_t)rows, 128, 64, 64) ||
-      !encode_tmap_2d_16bit(&m_edge, w.edge, 64, (uint64_t)(n_units * kM), 128, 64, 64))
-    return cudaErrorInvalidValue;
   bwd_prep_tc_kernel<<<(unsigned)((N * 8 + 255) / 256), 256, 0, s>>>(
       (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, (const __nv_bfloat16*)dout,
       (const __nv_bfloat16*)out, (const __nv_bfloat16*)out_lo, D, w.x16, w.v16, w.g16, N);
-  inverse_perm_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(perm, w.inv, p.L, rows,
-                                                                      status);
   int grid = sm_count();
   if ((int64_t)grid > n_units) grid = (int)n_units;
   auto kern = p.causal ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
@@ -832,12 +797,12 @@ cudaError_t launch_attn_bwd_tc(const lsh_problem& p, const void* qk, const void*
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemBytes, s>>>(
       w.x16, w.v16, w.g16, perm, lse, D,
-      m_dv, m_dqk, m_edge, p.L, p.n_rounds, p.scale, p.scale * kLog2e, (int)n_units,
+      w.part_dv, w.part_dqk, w.edge, w.emap, p.L, p.n_rounds, p.scale, p.scale * kLog2e, (int)n_units,
       units_per_seg, status);
-  unsort_kernel<<<(unsigned)((N * 8 + 255) / 256), 256, 0, s>>>(
-      w.part_dv, w.part_dqk, w.edge, w.inv, lse, (const __nv_bfloat16*)dout, dqk, dv, p.L,
-      p.n_rounds, units_per_seg, N, status);
-  note_launch(4);
+  sum_rounds_kernel<<<(unsigned)((N * 8 + 255) / 256), 256, 0, s>>>(
+      w.part_dv, w.part_dqk, w.edge, w.emap, lse, (const __nv_bfloat16*)dout, dqk, dv, p.L,
+      p.n_rounds, n_units * kM, N, status);
+  note_launch(3);
   return cudaGetLastError();
 }
 

@@ -17,12 +17,12 @@
 //   warps 0-3  : producers — cp.async gathers of x and v rows through perm
 //                straight into the 128-byte-swizzled K-major layout of a
 //                5-slot ring (a unit's first pair also needs chunk 2p0-1,
-//                which goes to one of 3 rotating side buffers); each thread
-//                then converts its own pieces of v bf16 -> fp16 in place
-//                (exact for |values| < 65504); x stays bf16, whose products
-//                are exact in the Q K^T MMA too. Software-pipelined one job
-//                deep, with the next job's perm entries loaded a job ahead;
-//   warp 12    : TMEM allocation; one thread issues S = Q K^T (three
+//                which goes to one of 3 rotating side buffers). v arrives
+//                as an fp16 copy made before the launch (exact for
+//                |values| < 65504); x stays bf16, whose products are exact
+//                in the Q K^T MMA too. Software-pipelined one job deep, with
+//                the next job's perm entries loaded a job ahead;
+//   warp 12    : TMEM allocation; one elected lane issues S = Q K^T (three
 //                128x64x64 MMAs per pair into a double-buffered TMEM S) and
 //                O = P V with P read from TMEM (A operand) and V from shared
 //                memory (MN-major B operand);
@@ -128,21 +128,15 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 }
 
 // Thread t copies 16-byte pieces 4*(t&1)..+3 of row t>>1 of a chunk tile into
-// their 128-byte-swizzled places (bf16; converted later in place).
-__device__ __forceinline__ void issue_row(const __nv_bfloat16* __restrict__ src_row, uint8_t* tile,
+// their 128-byte-swizzled places.
+template <typename T16>
+__device__ __forceinline__ void issue_row(const T16* __restrict__ src_row, uint8_t* tile,
                                           int row, int half) {
   const uint32_t base = smem_u32(tile) + row * 128;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int ch = half * 4 + i;
     cp_async16(base + (((uint32_t)ch ^ (uint32_t)(row & 7)) << 4), src_row + ch * 8);
-  }
-}
-__device__ __forceinline__ void convert_row(uint8_t* tile, int row, int half) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int ch = half * 4 + i;
-    convert_piece_bf16_to_f16(tile + row * 128 + ((ch ^ (row & 7)) << 4));
   }
 }
 
@@ -160,7 +154,7 @@ __device__ __forceinline__ bool fwd_issue_s(FwdBar* bar, uint32_t tmem, uint32_t
                                             uint32_t pre0, const Job& jb, int nn, int pb,
                                             int n_chunks, volatile int* abort, int* status) {
   const int s = nn % kSlots, b = nn & 1;
-  if (!mbar_wait(&bar->slot_full[s], (uint32_t)(nn / kSlots) & 1u, abort, status)) return false;
+  if (!__all_sync(0xffffffffu, mbar_wait(&bar->slot_full[s], (uint32_t)(nn / kSlots) & 1u, abort, status))) return false;
   tc_fence_after();
   const uint32_t sl = slot0 + (uint32_t)(s * kSlotBytes) / 16;
   const uint32_t d = tmem + (uint32_t)b * kSCols;
@@ -194,7 +188,7 @@ __device__ __forceinline__ void fwd_issue_pv(uint32_t d, uint32_t pa, uint32_t v
 
 template <bool kCausal>
 __global__ void __launch_bounds__(kThreads, 1)
-attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __restrict__ v,
+attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __half* __restrict__ v,
                    const int32_t* __restrict__ perm, __half* __restrict__ opart,
                    float* __restrict__ lsepart, int L, int n_rounds, int64_t N, float scale_log2,
                    int n_units, int units_per_seg, int* status) {
@@ -264,10 +258,6 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
     int pend_slot = 0, pend_pre = -1;
     bool ok = true;
     auto publish = [&]() {
-      uint8_t* ps = slots + pend_slot * kSlotBytes;
-      if (pend_pre >= 0) convert_row(pres + pend_pre * kPreBytes + kTile, row, half);
-      convert_row(ps + 2 * kTile, row, half);
-      if (pend_odd) convert_row(ps + 3 * kTile, row, half);
       fence_proxy_async();
       mbar_arrive(&bar->slot_full[pend_slot]);
     };
@@ -296,7 +286,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
       pos_p = checked(pos_p);
       uint8_t* sl = slots + s * kSlotBytes;
       const __nv_bfloat16* xb = qk + bh * L * 64;
-      const __nv_bfloat16* vb = v + bh * L * 64;
+      const __half* vb = v + bh * L * 64;
       if (use_pre) {
         uint8_t* pb = pres + pb_idx * kPreBytes;
         if (half == 0) bar->kpos_pre[pb_idx][row] = pos_p;
@@ -330,7 +320,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
   } else if (wgi == 3) {
     // ------------------------------------------------ MMA issuer (warp 12)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
-    if (warp == 12 && lane == 0) {
+    if (warp == 12) {
       const uint32_t slot0 = smem_u32(slots) >> 4, pre0 = smem_u32(pres) >> 4;
       JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
       Job cur, nxt;
@@ -350,8 +340,8 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
           break;
         // O = P V for job n
         const int b = n & 1;
-        if (!mbar_wait(&bar->p_full[b], (uint32_t)(n / 2) & 1u, abort, status)) break;
-        if (n >= 2 && !mbar_wait(&bar->o_free[b], (uint32_t)(n / 2 - 1) & 1u, abort, status))
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar->p_full[b], (uint32_t)(n / 2) & 1u, abort, status))) break;
+        if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar->o_free[b], (uint32_t)(n / 2 - 1) & 1u, abort, status)))
           break;
         tc_fence_after();
         const int s = n % kSlots;
@@ -532,10 +522,17 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __
 
 }  // namespace
 
+bool launch_attn_fwd_tc_ok(const lsh_problem& p) {
+  if (p.dtype != LSH_BF16 || p.chunk != kM || !(p.scale > 0.f)) return false;
+  const int64_t n_units =
+      (int64_t)p.B * p.H * p.n_rounds * (((p.L / kM + 1) / 2 + kUnit - 1) / kUnit);
+  return n_units <= INT32_MAX;
+}
+
 cudaError_t launch_attn_fwd_tc(const lsh_problem& p, const void* qk, const void* v,
                                const int32_t* perm, void* opart_f16, float* lsepart, int* status,
                                cudaStream_t s) {
-  if (p.dtype != LSH_BF16 || p.chunk != kM || !(p.scale > 0.f)) return cudaErrorNotSupported;
+  if (!launch_attn_fwd_tc_ok(p)) return cudaErrorNotSupported;
   const int n_chunks = p.L / kM;
   const int n_pairs = (n_chunks + 1) / 2;
   const int units_per_seg = (n_pairs + kUnit - 1) / kUnit;
@@ -549,7 +546,7 @@ cudaError_t launch_attn_fwd_tc(const lsh_problem& p, const void* qk, const void*
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemBytes, s>>>((const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, perm,
+  kern<<<grid, kThreads, kSmemBytes, s>>>((const __nv_bfloat16*)qk, (const __half*)v, perm,
                                           (__half*)opart_f16, lsepart, p.L, p.n_rounds, N,
                                           p.scale * kLog2e, (int)n_units, units_per_seg, status);
   note_launch();

@@ -18,6 +18,16 @@
 #include "internal.h"
 
 namespace lsh {
+// bf16 pair -> fp16 pair (exact inside the fp16 range)
+__device__ __forceinline__ uint32_t tc_bf16x2_to_f16x2(uint32_t u) {
+  const float lo = __uint_as_float(u << 16), hi = __uint_as_float(u & 0xffff0000u);
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+}  // namespace lsh
+
+namespace lsh {
 namespace {
 
 constexpr int kQ = 64;    // query rows per block
@@ -477,6 +487,17 @@ bwd_round_kernel(const T* __restrict__ qk, const T* __restrict__ v, const T* __r
 constexpr size_t kFwdSmem = (size_t)(2 * kQ + 2 * kK) * kP * 4 + (kQ + kK) * 4;
 constexpr size_t kBwdSmem = (size_t)(4 * kQ + 2 * kK) * kP * 4 + (kQ + kK) * 4 + 2 * kQ * 4;
 
+// fp16 copy of v for the tensor-core forward (exact inside the fp16 range;
+// outside it a value becomes inf, which the combine's check reports).
+__global__ void __launch_bounds__(256)
+v_to_f16_kernel(const __nv_bfloat16* __restrict__ v, __half* __restrict__ v16, int64_t n8) {
+  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= n8) return;
+  const uint4 w = __ldg(reinterpret_cast<const uint4*>(v) + k);
+  reinterpret_cast<uint4*>(v16)[k] = make_uint4(tc_bf16x2_to_f16x2(w.x), tc_bf16x2_to_f16x2(w.y),
+                                                tc_bf16x2_to_f16x2(w.z), tc_bf16x2_to_f16x2(w.w));
+}
+
 template <typename T>
 cudaError_t fwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* perm, T* out,
                   T* out_lo, float* lse, const FwdWs& ws, int* status, cudaStream_t s,
@@ -484,8 +505,17 @@ cudaError_t fwd_t(const lsh_problem& p, const T* qk, const T* v, const int32_t* 
   const int64_t N = (int64_t)p.B * p.H * p.L;
   const int64_t blocks = (int64_t)p.B * p.H * p.n_rounds * (p.L / kQ);
   const unsigned cblocks = (unsigned)((N * 16 + 255) / 256);
-  cudaError_t e = allow_tc ? launch_attn_fwd_tc(p, qk, v, perm, ws.opart, ws.lsepart, status, s)
-                           : cudaErrorNotSupported;
+  // the tensor-core forward reads an fp16 copy of v, kept in the unused half
+  // of the per-round output buffer (sized for fp32, filled with fp16; N is
+  // even, since L is a multiple of the chunk, so the copy ends inside it)
+  __half* v16 = (__half*)((char*)ws.opart + align_up((size_t)p.n_rounds * N * kD * 2, 256));
+  cudaError_t e = cudaErrorNotSupported;
+  if (allow_tc && launch_attn_fwd_tc_ok(p)) {
+    v_to_f16_kernel<<<(unsigned)((N * 8 + 255) / 256), 256, 0, s>>>(
+        (const __nv_bfloat16*)v, v16, N * 8);
+    note_launch();
+    e = launch_attn_fwd_tc(p, qk, v16, perm, ws.opart, ws.lsepart, status, s);
+  }
   if (e == cudaSuccess) {
     // the tensor-core forward handles bf16 problems only
     combine_f16_kernel<<<(unsigned)((N * 8 + 255) / 256), 256, 0, s>>>(

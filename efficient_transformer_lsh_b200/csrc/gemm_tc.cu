@@ -1,0 +1,305 @@
+// Dense products of the position-wise feed-forward layer that sits beside the
+// attention in a Reformer layer ("Reformer: The Efficient Transformer",
+// research.elamur.ai summary page, Key points, "Reversible layers": the
+// feed-forward layers run chunk by chunk) on the 5th-generation tensor cores:
+//
+//   C[M x N] = epilogue(A[M x K] B[K x N]),
+//
+// bf16 operands brought by TMA into 128-byte-swizzled shared memory, fp32
+// accumulation in TMEM. Each operand is read either K-major (stored
+// [rows][K]) or MN-major (stored [K][rows], i.e. the transpose of a stored
+// matrix, as the weight-gradient products need), from a plain row-major
+// matrix or from the attention's [B, H, L, 64] activation layout, in which
+// token row (b, l) has its 64 H features spread over the H head rows.
+//
+// One CTA computes one 128 x BN tile (BN = 64 or 128), K in steps of 64:
+//   warp 0     : one lane issues the TMA loads into a 4-stage ring;
+//   warp 1     : TMEM allocation; one lane issues the MMAs (128 x BN x 16);
+//   warps 2-5  : epilogue, one thread per tile row (TMEM lane): bias, ReLU,
+//                mask, residual, then bf16 or fp32 stores (optionally
+//                accumulating into fp32).
+// Every output element's K sum runs in the same order whichever tile or
+// launch computes its row, so splitting the rows into chunks does not change
+// a single bit of the result.
+#include <cuda_bf16.h>
+#include <stddef.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_common.cuh"
+#include "tma_host.h"
+
+namespace lsh {
+namespace {
+
+using namespace tc;
+
+constexpr int kBM = 128, kBK = 64, kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kATile = kBM * kBK * 2;   // 16 KB
+
+struct __align__(8) GemmBar {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int BN>
+constexpr size_t gemm_smem() {
+  return 1024 + (size_t)kStages * (kATile + BN * kBK * 2) + sizeof(GemmBar);
+}
+
+// Coordinates of the box whose first row is `row` (along the map's row
+// dimension) and whose 64 inner elements are block `blk` of the inner
+// dimension: plain maps are (cols, rows, 1, 1); head-layout maps are
+// (64, L, H, B) with token row r = b L + l and head h = blk.
+__device__ __forceinline__ void load_box(void* dst, const CUtensorMap* map, int heads, int L,
+                                         int64_t row, int blk, uint64_t* bar) {
+  if (heads)
+    tma_load_4d(dst, map, 0, (int32_t)(row % L), blk, (int32_t)(row / L), bar);
+  else
+    tma_load_4d(dst, map, blk * 64, (int32_t)row, 0, 0, bar);
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+               GemmOpDev a, GemmOpDev b, int K, GemmEpi e, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sa = smem;
+  uint8_t* sb = smem + kStages * kATile;
+  constexpr int kBTile = BN * kBK * 2;
+  GemmBar* bar = (GemmBar*)(sb + kStages * kBTile);
+  volatile int* abort = &bar->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * BN;
+  const int nk = K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bar->full[s], 1);
+      mbar_init(&bar->empty[s], 1);
+    }
+    mbar_init(&bar->acc_full, 1);
+    bar->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bar->tmem_base, BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+
+  if (warp == 0) {
+    // ---------------------------------------------- TMA producer
+    if (elect_one()) {
+      prefetch_tmap(&map_a);
+      prefetch_tmap(&map_b);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kStages;
+        if (kb >= kStages &&
+            !mbar_wait(&bar->empty[s], (uint32_t)(kb / kStages - 1) & 1u, abort, status))
+          break;
+        mbar_expect_tx(&bar->full[s], (uint32_t)(kATile + kBTile));
+        uint8_t* da = sa + s * kATile;
+        uint8_t* db = sb + s * kBTile;
+        if (a.mn_major) {
+          load_box(da, &map_a, a.heads, a.L, a.row0 + (int64_t)kb * kBK, m0 / 64, &bar->full[s]);
+          load_box(da + kATile / 2, &map_a, a.heads, a.L, a.row0 + (int64_t)kb * kBK, m0 / 64 + 1,
+                   &bar->full[s]);
+        } else {
+          load_box(da, &map_a, a.heads, a.L, a.row0 + m0, kb, &bar->full[s]);
+        }
+        if (b.mn_major) {
+#pragma unroll
+          for (int i = 0; i < BN / 64; ++i)
+            load_box(db + i * (64 * 128), &map_b, b.heads, b.L,
+                     b.row0 + (int64_t)kb * kBK, n0 / 64 + i, &bar->full[s]);
+        } else {
+          load_box(db, &map_b, b.heads, b.L, b.row0 + n0, kb, &bar->full[s]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------- MMA issuer
+    constexpr uint32_t kLboMN = desc_lbo(64 * 128);   // 64-wide M/N blocks, 8 KB apart
+    const uint32_t idesc = idesc_f16(kBM, BN, 1, a.mn_major != 0, b.mn_major != 0);
+    const uint32_t a_lbo = a.mn_major ? kLboMN : desc_lbo(16);
+    const uint32_t b_lbo = b.mn_major ? kLboMN : desc_lbo(16);
+    const uint32_t a_step = a.mn_major ? 128u : 2u;   // one K step of 16, in 16-byte units
+    const uint32_t b_step = b.mn_major ? 128u : 2u;
+    bool ok = true;
+    for (int kb = 0; kb < nk && ok; ++kb) {
+      const int s = kb % kStages;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&bar->full[s], (uint32_t)(kb / kStages) & 1u, abort, status));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t alo = (smem_u32(sa + s * kATile) >> 4) | a_lbo;
+      const uint32_t blo = (smem_u32(sb + s * kBTile) >> 4) | b_lbo;
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_ss_w(tmem, alo + a_step * ks, blo + b_step * ks, kDescHi1024, idesc,
+                 (kb > 0 || ks > 0) ? 1u : 0u);
+      mma_commit(&bar->empty[s]);
+    }
+    mma_commit(&bar->acc_full);
+  } else {
+    // ---------------------------------------------- epilogue
+    const int q = warp & 3;              // TMEM lane quarter of this warp
+    const int r = q * 32 + lane;         // tile row
+    const int64_t row = (int64_t)m0 + r;
+    const bool got = __all_sync(0xffffffffu, mbar_wait(&bar->acc_full, 0u, abort, status));
+    tc_fence_after();
+    const bool live = got && row < e.M;
+    const int64_t orow = e.row0 + row;
+    // element offset of (orow, column c) in the output / residual layout
+    auto out_off = [&](int c) -> int64_t {
+      if (e.out_heads) {
+        const int64_t bb = orow / e.L, l = orow - bb * e.L;
+        return ((bb * e.H + c / 64) * e.L + l) * 64 + (c & 63);
+      }
+      return orow * e.ldo + c;
+    };
+    if (got) {
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t acc[16];
+        tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, acc);
+        tmem_ld_wait();
+        if (!live) continue;
+        const int c = n0 + c0;
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(acc[i]);
+        if (e.bias) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] += __ldg(e.bias + c + i);
+        }
+        if (e.relu) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = fmaxf(v[i], 0.f);
+        }
+        if (e.mask) {
+          const uint4* mp = reinterpret_cast<const uint4*>(e.mask + row * e.ldm + c);
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const uint4 w = __ldg(mp + k);
+            const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              if (!(__uint_as_float(u[i] << 16) > 0.f)) v[8 * k + 2 * i] = 0.f;
+              if (!(__uint_as_float(u[i] & 0xffff0000u) > 0.f)) v[8 * k + 2 * i + 1] = 0.f;
+            }
+          }
+        }
+        const int64_t off = out_off(c);
+        if (e.res) {
+          const uint4* rp = reinterpret_cast<const uint4*>(e.res + off);
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const uint4 w = __ldg(rp + k);
+            const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              v[8 * k + 2 * i] = fmaf(e.res_sign, v[8 * k + 2 * i], __uint_as_float(u[i] << 16));
+              v[8 * k + 2 * i + 1] =
+                  fmaf(e.res_sign, v[8 * k + 2 * i + 1], __uint_as_float(u[i] & 0xffff0000u));
+            }
+          }
+        }
+        if (e.out_f32) {
+          float4* op = reinterpret_cast<float4*>((float*)e.out + off);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float4 o = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            if (e.accumulate) {
+              const float4 p = op[k];
+              o.x += p.x;
+              o.y += p.y;
+              o.z += p.z;
+              o.w += p.w;
+            }
+            op[k] = o;
+          }
+        } else {
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          uint4* op = reinterpret_cast<uint4*>((__nv_bfloat16*)e.out + off);
+          op[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          op[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+}
+
+// Tensor map of one operand: plain (cols, rows, 1, 1) or head layout
+// (64, L, H, B); box of 64 inner elements by `box_rows` rows.
+bool encode_op(CUtensorMap* map, const GemmOpHost& o, uint32_t box_rows) {
+  uint64_t dims[4], strides[3];
+  const uint32_t box[4] = {64, box_rows, 1, 1};
+  if (o.heads) {
+    dims[0] = 64;
+    dims[1] = (uint64_t)o.L;
+    dims[2] = (uint64_t)o.H;
+    dims[3] = (uint64_t)o.B;
+    strides[0] = 128;
+    strides[1] = (uint64_t)o.L * 128;
+    strides[2] = (uint64_t)o.H * o.L * 128;
+  } else {
+    dims[0] = (uint64_t)o.cols;
+    dims[1] = (uint64_t)o.rows;
+    dims[2] = 1;
+    dims[3] = 1;
+    strides[0] = (uint64_t)o.cols * 2;
+    strides[1] = strides[0] * (uint64_t)o.rows;
+    strides[2] = strides[1];
+  }
+  return encode_tmap_4d_16bit(map, o.base, dims, strides, box);
+}
+
+template <int BN>
+cudaError_t launch_bn(const GemmOpHost& a, const GemmOpHost& b, int M, int N, int K,
+                      const GemmEpi& e, int* status, cudaStream_t s) {
+  CUtensorMap ma, mb;
+  if (!encode_op(&ma, a, a.mn_major ? 64 : kBM) || !encode_op(&mb, b, b.mn_major ? 64 : BN))
+    return cudaErrorInvalidValue;
+  const GemmOpDev da{a.mn_major, a.heads, a.L, a.row0};
+  const GemmOpDev db{b.mn_major, b.heads, b.L, b.row0};
+  constexpr size_t smem = gemm_smem<BN>();
+  cudaError_t err =
+      cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  const dim3 grid((unsigned)((M + kBM - 1) / kBM), (unsigned)(N / BN));
+  gemm_tc_kernel<BN><<<grid, kThreads, smem, s>>>(ma, mb, da, db, K, e, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(const GemmOpHost& a, const GemmOpHost& b, int M, int N, int K,
+                           const GemmEpi& e, int* status, cudaStream_t s) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % kBK != 0 || N % 64 != 0) return cudaErrorInvalidValue;
+  if (N % 128 == 0) return launch_bn<128>(a, b, M, N, K, e, status, s);
+  return launch_bn<64>(a, b, M, N, K, e, status, s);
+}
+
+}  // namespace lsh

@@ -190,7 +190,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ---------------- MMA issuer ----------------
       // Tiles alternate between the two accumulators / epilogue warpgroups;
       // the chunks of a pair of tiles are interleaved so both stay busy, and
@@ -200,20 +200,20 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
       int uses0 = 0, uses1 = 0, rb = 0;
       bool ok = true;
       if (!stream_r) {
-        ok = mbar_wait(&bar->r_full[0], 0u, abort, status);
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar->r_full[0], 0u, abort, status));
         rb = 1;
       }
       for (int it0 = 0; it0 < n_mine && ok; it0 += 2) {
         const int cnt = min(2, n_mine - it0);
         for (int k = 0; k < cnt && ok; ++k)
-          ok = mbar_wait(&bar->x_full[(it0 + k) % kStages], (uint32_t)((it0 + k) / kStages) & 1u,
-                         abort, status);
+          ok = __all_sync(0xffffffffu, mbar_wait(&bar->x_full[(it0 + k) % kStages], (uint32_t)((it0 + k) / kStages) & 1u,
+                         abort, status));
         if (!ok) break;
         tc_fence_after();
         for (int b = 0; b < n_blk && ok; ++b) {
           const int rs = stream_r ? rb % kRStages : 0;
           if (stream_r) {
-            ok = mbar_wait(&bar->r_full[rs], (uint32_t)(rb / kRStages) & 1u, abort, status);
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar->r_full[rs], (uint32_t)(rb / kRStages) & 1u, abort, status));
             if (!ok) break;
             tc_fence_after();
           }
@@ -224,7 +224,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
               const int it = it0 + k, w = it & 1, s = it % kStages;
               int& uses = w ? uses1 : uses0;
               if (uses > 0 &&
-                  !mbar_wait(&bar->acc_empty[w], (uint32_t)(uses - 1) & 1u, abort, status)) {
+                  !__all_sync(0xffffffffu, mbar_wait(&bar->acc_empty[w], (uint32_t)(uses - 1) & 1u, abort, status))) {
                 ok = false;
                 break;
               }

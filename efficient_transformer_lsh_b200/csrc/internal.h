@@ -50,14 +50,15 @@ cudaError_t launch_attn_fwd(const lsh_problem& p, const void* qk, const void* v,
 
 // tcgen05 per-round forward (bf16, chunk 64): writes fp16 per-round outputs
 // [n_rounds][B*H*L][64] and lse_r; cudaErrorNotSupported for other shapes.
-cudaError_t launch_attn_fwd_tc(const lsh_problem& p, const void* qk, const void* v,
+bool launch_attn_fwd_tc_ok(const lsh_problem& p);
+cudaError_t launch_attn_fwd_tc(const lsh_problem& p, const void* qk, const void* v16,
                                const int32_t* perm, void* opart_f16, float* lsepart, int* status,
                                cudaStream_t s);
 
 // tcgen05 backward (bf16, chunk 64): forms D = dout . (out + out_lo) into D
 // and fp16 copies of qk, v, dout, then writes dqk and dv (every element, the
 // self-attending rows' dout included); `ws` holds bwd_tc_ws_bytes(p) bytes
-// (fp16 copies, inverse permutation, per-round fp16 partials).
+// (fp16 copies, per-round fp16 partials in token order, edge map).
 // bwd_tc_ws_bytes is 0 and the launcher returns cudaErrorNotSupported for
 // other problems.
 size_t bwd_tc_ws_bytes(const lsh_problem& p);
@@ -82,6 +83,44 @@ cudaError_t launch_local_bwd(const lsh_problem& p, int n_back, int n_fwd, const 
                              const void* v, const void* out, const void* out_lo, const float* lse,
                              const void* dout, float* dqk, float* dv, void* ws, int* status,
                              cudaStream_t s);
+
+// ---- dense products of the feed-forward layer (tcgen05) -------------------
+// An operand of C = A B: mn_major = stored [K][rows] (else [rows][K]); heads =
+// the attention's [B, H, L, 64] layout read as token rows b L + l with 64 H
+// columns (else a plain row-major matrix of rows x cols); row0 = first row
+// (tokens for the head layout, K rows when mn_major) of this product.
+struct GemmOpDev {
+  int mn_major, heads, L;
+  int64_t row0;
+};
+struct GemmOpHost {
+  const void* base;
+  int mn_major, heads;
+  int64_t rows, cols;   // plain matrix extent
+  int L, H, B;          // head layout extent
+  int64_t row0;
+};
+// Epilogue, per element (row, column c) of the M x N result:
+//   v = acc + bias[c]; v = max(v, 0) if relu; v = 0 unless mask[row][c] > 0;
+//   v = res + res_sign * v where res is given (same layout as the output);
+//   out (bf16, or fp32 with optional accumulate) at row0 + row.
+struct GemmEpi {
+  const float* bias;
+  int relu;
+  const __nv_bfloat16* mask;
+  int64_t ldm;
+  const __nv_bfloat16* res;
+  float res_sign;
+  void* out;
+  int out_f32, accumulate, out_heads;
+  int64_t ldo, row0;
+  int L, H;
+  int M;
+};
+// K a multiple of 64, N a multiple of 64; rows past M are neither read into
+// the output nor written.
+cudaError_t launch_gemm_tc(const GemmOpHost& a, const GemmOpHost& b, int M, int N, int K,
+                           const GemmEpi& e, int* status, cudaStream_t s);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

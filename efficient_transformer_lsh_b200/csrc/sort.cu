@@ -9,12 +9,14 @@
 //  * n_buckets <= 8192 (every shape the workloads use): two kernels over
 //    blocks of 8K-32K consecutive positions, one CTA each (see the counting
 //    path below): block totals per bucket from shared-memory atomics, then a
-//    scatter kernel that forms the bucket bases itself and ranks positions
-//    within each warp step by ballots over the bucket bits;
+//    scatter kernel that ranks positions within each warp step by a warp
+//    bitonic sort of (bucket, lane) keys; the bucket bases come from the
+//    scatter kernel itself, or, for many blocks or few segments, from two
+//    small scan kernels;
 //  * larger bucket counts: per 4096-position tile the packed keys
 //    (bucket << 12 | local index) are sorted in shared memory by a bitonic
 //    network; row_scan / bucket_scan form the bases; scatter places them.
-// Ranks follow position order inside a warp step (lane order),
+// Ranks follow position order inside a warp step (the lane breaks ties),
 // across the steps of a warp (in order), across the warps of a block
 // (exclusive prefix of their counts) and across blocks (counts of the blocks
 // before), so the whole sort is stable.
@@ -187,12 +189,16 @@ scatter_kernel(const uint32_t* __restrict__ sorted, const int32_t* __restrict__ 
 //   sort_scatter_kernel: bucket bases of the segment (exclusive scan of the
 //                        totals over buckets) plus the counts of the blocks
 //                        before q; then each warp takes its positions 32 at a
-//                        time and finds, with one ballot per bucket bit, the
-//                        lanes that share each lane's bucket: a position's rank
-//                        is the number of such lanes below it. A first pass
-//                        counts per warp, an exclusive prefix over warps gives
-//                        each warp's run, and a second pass places every
-//                        position at its slot.
+//                        time, sorts the 32 (bucket, lane) keys with a warp
+//                        bitonic network so equal buckets form contiguous
+//                        segments in lane order, and ranks each position
+//                        within its segment. A first pass counts per warp, an
+//                        exclusive prefix over warps gives each warp's run, and
+//                        a second pass places every position at its slot.
+//   sort_qscan_kernel,
+//   sort_bscan_kernel:   (when Q * n_buckets is large or S * Q small) the
+//                        prefix over blocks and the bucket bases, so that the
+//                        scatter kernel reads two numbers per bucket.
 constexpr int kWarpMaxBuckets = 8192;
 constexpr int kSortSmemBudget = 200 * 1024;
 
@@ -241,18 +247,44 @@ __device__ __forceinline__ uint32_t load_bucket(const int32_t* __restrict__ seg_
   return b;
 }
 
-// The lanes of the warp whose bucket equals this lane's: one ballot per bucket
-// bit (nbits of them), each lane keeping the lanes that agree on the bit.
-// Lanes past the end of the segment (bucket 0xffffffff) are excluded.
-__device__ __forceinline__ uint32_t same_bucket_lanes(uint32_t b, int nbits) {
-  const bool live = b != 0xffffffffu;
-  uint32_t eq = __ballot_sync(0xffffffffu, live);
-  for (int k = 0; k < nbits; ++k) {
-    const bool bit = (b >> k) & 1u;
-    const uint32_t m = __ballot_sync(0xffffffffu, bit);
-    eq &= bit ? m : ~m;
+// Sorts the warp's 32 keys ascending (bitonic network over lanes).
+__device__ __forceinline__ uint32_t warp_sort32(uint32_t key, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint32_t o = __shfl_xor_sync(0xffffffffu, key, j);
+      const bool up = (lane & k) == 0, lower = (lane & j) == 0;
+      key = (lower == up) ? min(key, o) : max(key, o);
+    }
   }
-  return eq;
+  return key;
+}
+
+// One step of 32 positions: after sorting (bucket << 5 | lane) keys, lane k
+// holds sorted entry k: its bucket, the lane (position offset) it came from,
+// its rank among the entries of its bucket, and whether it ends the bucket's
+// segment (then `len` is the segment's length).
+struct StepRank {
+  uint32_t bucket;
+  int src, rank, len;
+  bool live, last;
+};
+__device__ __forceinline__ StepRank rank_step(uint32_t b, int lane) {
+  const uint32_t key = warp_sort32(b == 0xffffffffu ? 0xffffffffu : (b << 5) | (uint32_t)lane, lane);
+  StepRank r;
+  r.live = key != 0xffffffffu;
+  r.bucket = key >> 5;
+  r.src = (int)(key & 31u);
+  const uint32_t prev = __shfl_up_sync(0xffffffffu, r.bucket, 1);
+  const uint32_t next = __shfl_down_sync(0xffffffffu, r.bucket, 1);
+  const bool first = lane == 0 || prev != r.bucket;
+  r.last = lane == 31 || next != r.bucket;
+  const uint32_t starts = __ballot_sync(0xffffffffu, first);
+  const int seg0 = 31 - __clz(starts & (0xffffffffu >> (31 - lane)));
+  r.rank = lane - seg0;
+  r.len = r.rank + 1;
+  return r;
 }
 
 __global__ void __launch_bounds__(1024)
@@ -381,14 +413,11 @@ sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restric
   const int32_t* sbk = bucket + seg * L;
   const int64_t i0 = (int64_t)q * P + (int64_t)w * PW;
   uint16_t* mine = cnt + w * n_buckets;
-  const int nbits = 32 - __clz(n_buckets - 1);
-  const uint32_t below = (1u << lane) - 1u;
-  // pass 1: this warp's count of every bucket (the lowest lane of each group
-  // of equal buckets adds the group's size)
+  // pass 1: this warp's count of every bucket
   for (int st = 0; st < PW; st += 32) {
     const uint32_t b = load_bucket(sbk, i0 + st + lane, L, n_buckets, nullptr);
-    const uint32_t eq = same_bucket_lanes(b, nbits);
-    if (b != 0xffffffffu && (eq & below) == 0u) mine[b] = (uint16_t)(mine[b] + __popc(eq));
+    const StepRank r = rank_step(b, lane);
+    if (r.live && r.last) mine[r.bucket] = (uint16_t)(mine[r.bucket] + r.len);
     __syncwarp();
   }
   __syncthreads();
@@ -406,10 +435,10 @@ sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restric
   int32_t* out = perm + seg * L;
   for (int st = 0; st < PW; st += 32) {
     const uint32_t b = load_bucket(sbk, i0 + st + lane, L, n_buckets, nullptr);
-    const uint32_t eq = same_bucket_lanes(b, nbits);
-    if (b != 0xffffffffu) out[base[b] + mine[b] + __popc(eq & below)] = (int32_t)(i0 + st + lane);
+    const StepRank r = rank_step(b, lane);
+    if (r.live) out[base[r.bucket] + mine[r.bucket] + r.rank] = (int32_t)(i0 + st + r.src);
     __syncwarp();
-    if (b != 0xffffffffu && (eq & below) == 0u) mine[b] = (uint16_t)(mine[b] + __popc(eq));
+    if (r.live && r.last) mine[r.bucket] = (uint16_t)(mine[r.bucket] + r.len);
     __syncwarp();
   }
 }

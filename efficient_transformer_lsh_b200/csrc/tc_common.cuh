@@ -124,6 +124,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       "l"((uint64_t)map), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
+// 4D tiled load (coordinates innermost first); completion counted on `bar`.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int32_t c0,
+                                            int32_t c1, int32_t c2, int32_t c3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
 }
@@ -159,6 +168,13 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int32_t x, 
 }
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Untiled bulk copy of `bytes` (a multiple of 16) from shared to global
+// memory, both addresses 16-byte aligned; tracked in this thread's bulk groups.
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(ssrc), "r"(bytes)
+               : "memory");
 }
 // Waits until the shared-memory sources of all committed bulk groups have been read.
 __device__ __forceinline__ void bulk_wait_read_all() {
@@ -287,6 +303,15 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int ab_type, bool
          | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// One lane of a converged warp (the lowest active one).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // D[tmem] (+)= A * B, issued by one thread, with each shared-memory
 // descriptor given as its two 32-bit words: lo = (address >> 4) | (LBO >> 4)
 // << 16, hi = the SBO / version / swizzle word (smem_desc's upper half).
@@ -297,7 +322,7 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int ab_type, bool
 // half), B in shared memory.
 __device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
                                          uint32_t hi, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
+  if (elect_one()) asm volatile(
       "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
       "setp.ne.b32 p, %5, 0;\n\t"
       "mov.b64 da, {%1, %3};\n\t"
@@ -307,7 +332,7 @@ __device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint32_t a_lo, uint32_
 }
 __device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
                                          uint32_t hi, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
+  if (elect_one()) asm volatile(
       "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
       "setp.ne.b32 p, %5, 0;\n\t"
       "mov.b64 db, {%2, %3};\n\t"
@@ -321,7 +346,7 @@ __host__ __device__ constexpr uint32_t desc_lbo(uint32_t lbo_bytes) { return ((l
 
 // Arrives on `bar` once every previously issued MMA of this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile(
+  if (elect_one()) asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_u32(bar))
       : "memory");

@@ -40,6 +40,20 @@ bool encode_tmap_2d_16bit(CUtensorMap* map, const void* base, uint64_t inner, ui
   return r == CUDA_SUCCESS;
 }
 
+bool encode_tmap_4d_16bit(CUtensorMap* map, const void* base, const uint64_t dims[4],
+                          const uint64_t strides[3], const uint32_t box[4]) {
+  EncodeFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[4] = {dims[0], dims[1], dims[2], dims[3]};
+  cuuint64_t st[3] = {strides[0], strides[1], strides[2]};
+  cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), d, st, bx,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int sm_count() {
   static int cache[64] = {};
   int dev = 0;

@@ -136,10 +136,10 @@ lsh_status lsh_attn_fwd(const lsh_problem* p, const void* qk, const void* v,
  *   inputs; out_lo may be NULL, in which case D is formed from `out` alone
  *   (for bf16 problems that adds the rounding error of out to D).
  *   Workspace: D (4 bytes per token) and, for the tensor-core path (bf16,
- *   chunk 64), the inverse permutation (4 bytes per token and round) and the
- *   per-round fp16 partial gradients in sorted order (256 bytes per token and
- *   round), about 260 bytes per token and round in all. dqk and dv are
- *   overwritten, not accumulated into.
+ *   chunk 64), fp16 copies of qk, v and dout (384 bytes per token), the
+ *   per-round fp16 partial gradients in token order (256 bytes per token and
+ *   round) and a map of the partial rows at work-unit edges (4 bytes per
+ *   token and round). dqk and dv are overwritten, not accumulated into.
  */
 size_t lsh_bwd_workspace_size(const lsh_problem* p);
 lsh_status lsh_attn_bwd(const lsh_problem* p, const void* qk, const void* v,
