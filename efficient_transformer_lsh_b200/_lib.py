@@ -23,7 +23,9 @@ EXPORTS = ("lsh_hash", "lsh_sort_workspace_size", "lsh_sort", "lsh_fwd_workspace
            "lsh_attn_fwd", "lsh_bwd_workspace_size", "lsh_attn_bwd", "lsh_device_status",
            "lsh_status_string", "lsh_launch_count", "lsh_sort_noalloc", "lsh_check_wait_timeout",
            "lsh_local_fwd_workspace_size", "lsh_local_attn_fwd", "lsh_local_bwd_workspace_size",
-           "lsh_local_attn_bwd")
+           "lsh_local_attn_bwd", "lsh_ff_workspace_size", "lsh_ff_fwd", "lsh_ff_bwd",
+           "lsh_rev_fwd_workspace_size", "lsh_rev_fwd", "lsh_rev_bwd_workspace_size",
+           "lsh_rev_bwd")
 # Size of the library-owned scratch used by lsh_sort_noalloc (matches lsh.h).
 SORT_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -45,6 +47,15 @@ class lsh_problem(ctypes.Structure):
                 ("causal", ctypes.c_int32), ("scale", ctypes.c_float), ("dtype", ctypes.c_int32)]
 
 
+class lsh_ff_problem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("L", ctypes.c_int32),
+                ("d_ff", ctypes.c_int32), ("ff_chunk", ctypes.c_int32)]
+
+
+def make_ff_problem(B, H, L, d_ff, ff_chunk) -> lsh_ff_problem:
+    return lsh_ff_problem(int(B), int(H), int(L), int(d_ff), int(ff_chunk))
+
+
 def make_problem(B, H, L, d, n_buckets, n_rounds, chunk, causal, scale, dtype) -> lsh_problem:
     if isinstance(dtype, str):
         dtype = {"f32": LSH_F32, "bf16": LSH_BF16}[dtype]
@@ -63,6 +74,7 @@ def lib() -> ctypes.CDLL:
                 f"{LIB_PATH} is missing: build it with `python -m efficient_transformer_lsh_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
         P = ctypes.POINTER(lsh_problem)
+        F = ctypes.POINTER(lsh_ff_problem)
         vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
         sig = {
             "lsh_hash": ([P, vp, vp, vp, vp], ctypes.c_int),
@@ -82,6 +94,13 @@ def lib() -> ctypes.CDLL:
             "lsh_local_bwd_workspace_size": ([P, i32, i32], sz),
             "lsh_local_attn_bwd": ([P, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
                                    ctypes.c_int),
+            "lsh_ff_workspace_size": ([F], sz),
+            "lsh_ff_fwd": ([F] + [vp] * 8 + [sz, vp], ctypes.c_int),
+            "lsh_ff_bwd": ([F] + [vp] * 15 + [sz, vp], ctypes.c_int),
+            "lsh_rev_fwd_workspace_size": ([P, F], sz),
+            "lsh_rev_fwd": ([P, F] + [vp] * 11 + [sz, vp], ctypes.c_int),
+            "lsh_rev_bwd_workspace_size": ([P, F], sz),
+            "lsh_rev_bwd": ([P, F] + [vp] * 18 + [sz, vp], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -179,6 +198,48 @@ def lsh_local_attn_bwd(p: lsh_problem, n_back, n_fwd, qk, v, out, out_lo, lse, d
                                     _ptr(out), _ptr(out_lo), _ptr(lse), _ptr(dout), _ptr(dqk),
                                     _ptr(dv), _ptr(ws), int(ws_bytes), _stream(stream)),
            "lsh_local_attn_bwd")
+
+
+def lsh_ff_workspace_size(f: lsh_ff_problem) -> int:
+    return int(lib().lsh_ff_workspace_size(ctypes.byref(f)))
+
+
+def lsh_ff_fwd(f: lsh_ff_problem, x, W1, b1, W2, b2, res, y, ws, ws_bytes: int, stream=None):
+    _check(lib().lsh_ff_fwd(ctypes.byref(f), _ptr(x), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2),
+                            _ptr(res), _ptr(y), _ptr(ws), int(ws_bytes), _stream(stream)),
+           "lsh_ff_fwd")
+
+
+def lsh_ff_bwd(f: lsh_ff_problem, x, W1, b1, W2, b2, dy, dres, y_in, rec, dx, dW1, db1, dW2, db2,
+               ws, ws_bytes: int, stream=None):
+    _check(lib().lsh_ff_bwd(ctypes.byref(f), _ptr(x), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2),
+                            _ptr(dy), _ptr(dres), _ptr(y_in), _ptr(rec), _ptr(dx), _ptr(dW1),
+                            _ptr(db1), _ptr(dW2), _ptr(db2), _ptr(ws), int(ws_bytes),
+                            _stream(stream)), "lsh_ff_bwd")
+
+
+def lsh_rev_fwd_workspace_size(p: lsh_problem, f: lsh_ff_problem) -> int:
+    return int(lib().lsh_rev_fwd_workspace_size(ctypes.byref(p), ctypes.byref(f)))
+
+
+def lsh_rev_fwd(p: lsh_problem, f: lsh_ff_problem, x1, x2, R, W1, b1, W2, b2, y1, y2, perm, ws,
+                ws_bytes: int, stream=None):
+    _check(lib().lsh_rev_fwd(ctypes.byref(p), ctypes.byref(f), _ptr(x1), _ptr(x2), _ptr(R),
+                             _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(y1), _ptr(y2),
+                             _ptr(perm), _ptr(ws), int(ws_bytes), _stream(stream)), "lsh_rev_fwd")
+
+
+def lsh_rev_bwd_workspace_size(p: lsh_problem, f: lsh_ff_problem) -> int:
+    return int(lib().lsh_rev_bwd_workspace_size(ctypes.byref(p), ctypes.byref(f)))
+
+
+def lsh_rev_bwd(p: lsh_problem, f: lsh_ff_problem, y1, y2, dy1, dy2, perm, W1, b1, W2, b2, x1, x2,
+                dx1, dx2, dW1, db1, dW2, db2, ws, ws_bytes: int, stream=None):
+    _check(lib().lsh_rev_bwd(ctypes.byref(p), ctypes.byref(f), _ptr(y1), _ptr(y2), _ptr(dy1),
+                             _ptr(dy2), _ptr(perm), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2),
+                             _ptr(x1), _ptr(x2), _ptr(dx1), _ptr(dx2), _ptr(dW1), _ptr(db1),
+                             _ptr(dW2), _ptr(db2), _ptr(ws), int(ws_bytes), _stream(stream)),
+           "lsh_rev_bwd")
 
 
 def lsh_device_status(stream=None) -> int:

@@ -121,6 +121,57 @@ class LocalAttention:
         return self.dqk, self.dv
 
 
+class ReversibleLSHBlock:
+    """Reversible residual block y1 = x1 + F(x2), y2 = x2 + G(y1) with F the
+    LSH attention of x2 (qk = v = x2) and G the chunked feed-forward
+    max(0, x W1 + b1) W2 + b2, for one fixed shape. The backward rebuilds
+    x1, x2 from y1, y2 (nothing of the forward is kept but the sort
+    permutation). Activations and their gradients [B, H, L, 64] bf16
+    (d_model = 64 H); W1 [64 H, d_ff], W2 [d_ff, 64 H] bf16; b1, b2 and the
+    weight gradients float32."""
+
+    def __init__(self, B, H, L, n_buckets, n_rounds, chunk, causal, d_ff, ff_chunk,
+                 scale: Optional[float] = None, device="cuda"):
+        if scale is None:
+            scale = 1.0 / 8.0
+        self.p = _lib.make_problem(B, H, L, 64, n_buckets, n_rounds, chunk, causal, scale, "bf16")
+        self.f = _lib.make_ff_problem(B, H, L, d_ff, ff_chunk)
+        self.shape = (B, H, L, 64)
+        dev = torch.device(device)
+        D = 64 * H
+        self.perm = torch.empty((B, H, n_rounds, L), dtype=torch.int32, device=dev)
+        self.y1 = torch.empty(self.shape, dtype=torch.bfloat16, device=dev)
+        self.y2 = torch.empty_like(self.y1)
+        self.x1 = torch.empty_like(self.y1)
+        self.x2 = torch.empty_like(self.y1)
+        self.dx1 = torch.empty_like(self.y1)
+        self.dx2 = torch.empty_like(self.y1)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.dW1 = torch.empty((D, d_ff), **f32)
+        self.db1 = torch.empty((d_ff,), **f32)
+        self.dW2 = torch.empty((d_ff, D), **f32)
+        self.db2 = torch.empty((D,), **f32)
+        self.ws_fwd_bytes = _lib.lsh_rev_fwd_workspace_size(self.p, self.f)
+        self.ws_bwd_bytes = _lib.lsh_rev_bwd_workspace_size(self.p, self.f)
+        if min(self.ws_fwd_bytes, self.ws_bwd_bytes) == 0 and B * H * L > 0:
+            raise _lib.LshError(1, "workspace size query (problem rejected)")
+        u8 = dict(dtype=torch.uint8, device=dev)
+        self.ws_fwd = torch.empty(max(1, self.ws_fwd_bytes), **u8)
+        self.ws_bwd = torch.empty(max(1, self.ws_bwd_bytes), **u8)
+
+    def forward(self, x1, x2, R, W1, b1, W2, b2, stream=None):
+        _lib.lsh_rev_fwd(self.p, self.f, x1, x2, R, W1, b1, W2, b2, self.y1, self.y2, self.perm,
+                         self.ws_fwd, self.ws_fwd_bytes, stream)
+        return self.y1, self.y2
+
+    def backward(self, y1, y2, dy1, dy2, W1, b1, W2, b2, stream=None):
+        """Returns (x1, x2, dx1, dx2, dW1, db1, dW2, db2)."""
+        _lib.lsh_rev_bwd(self.p, self.f, y1, y2, dy1, dy2, self.perm, W1, b1, W2, b2, self.x1,
+                         self.x2, self.dx1, self.dx2, self.dW1, self.db1, self.dW2, self.db2,
+                         self.ws_bwd, self.ws_bwd_bytes, stream)
+        return self.x1, self.x2, self.dx1, self.dx2, self.dW1, self.db1, self.dW2, self.db2
+
+
 class _LSHAttentionFn(torch.autograd.Function):
     @staticmethod
     def forward(ctx, qk, v, R, runner: LSHAttention):

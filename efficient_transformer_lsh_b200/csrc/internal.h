@@ -1,6 +1,7 @@
 // Host-side interface between the C ABI (lsh_api.cu) and the kernel files.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -123,5 +124,26 @@ cudaError_t launch_gemm_tc(const GemmOpHost& a, const GemmOpHost& b, int M, int 
                            const GemmEpi& e, int* status, cudaStream_t s);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---- chunked feed-forward and the reversible block (rev_block.cu) ----------
+size_t ff_ws_bytes(const lsh_ff_problem& f);
+cudaError_t launch_ff_fwd(const lsh_ff_problem& f, const void* x, const void* W1, const float* b1,
+                          const void* W2, const float* b2, const void* res, void* y, void* ws,
+                          int* status, cudaStream_t s);
+cudaError_t launch_ff_bwd(const lsh_ff_problem& f, const void* x, const void* W1, const float* b1,
+                          const void* W2, const float* b2, const void* dy, const void* dres,
+                          const void* y_in, void* rec, void* dx, float* dW1, float* db1,
+                          float* dW2, float* db2, void* ws, int* status, cudaStream_t s);
+size_t rev_fwd_ws_bytes(const lsh_problem& p, const lsh_ff_problem& f);
+size_t rev_bwd_ws_bytes(const lsh_problem& p, const lsh_ff_problem& f);
+cudaError_t launch_rev_fwd(const lsh_problem& p, const lsh_ff_problem& f, const void* x1,
+                           const void* x2, const void* R, const void* W1, const float* b1,
+                           const void* W2, const float* b2, void* y1, void* y2, int32_t* perm,
+                           void* ws, int* status, cudaStream_t s);
+cudaError_t launch_rev_bwd(const lsh_problem& p, const lsh_ff_problem& f, const void* y1,
+                           const void* y2, const void* dy1, const void* dy2, const int32_t* perm,
+                           const void* W1, const float* b1, const void* W2, const float* b2,
+                           void* x1, void* x2, void* dx1, void* dx2, float* dW1, float* db1,
+                           float* dW2, float* db2, void* ws, int* status, cudaStream_t s);
 
 }  // namespace lsh

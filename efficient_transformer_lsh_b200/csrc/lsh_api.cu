@@ -1,6 +1,7 @@
 // C ABI of the LSH-attention library: argument checks, workspace sizing,
 // dispatch to the kernels, and the device status word.
 #include <atomic>
+#include <initializer_list>
 #include <cmath>
 #include <mutex>
 
@@ -206,6 +207,113 @@ lsh_status lsh_local_attn_bwd(const lsh_problem* p, int32_t n_back, int32_t n_fw
   if (p->dtype == LSH_F32) out_lo = nullptr;
   return cuda_status(launch_local_bwd(*p, n_back, n_fwd, qk, v, out, out_lo, lse, dout, dqk, dv,
                                       ws, device_status_word(), (cudaStream_t)stream));
+}
+
+static lsh_status check_ff(const lsh_ff_problem* f) {
+  if (!f) return LSH_ERR_INVALID_ARG;
+  if (f->B < 0 || f->H < 1 || f->L < 0 || f->d_ff < 128 || f->ff_chunk < 128)
+    return LSH_ERR_INVALID_ARG;
+  if (f->L % 128 != 0 || f->d_ff % 128 != 0 || f->ff_chunk % 128 != 0) return LSH_ERR_INVALID_ARG;
+  if (f->d_ff > 65536 || 64 * (int64_t)f->H > 65536) return LSH_ERR_UNSUPPORTED;
+  if ((int64_t)f->B * f->H * f->L * 64 > (int64_t)INT32_MAX * 64 ||
+      (int64_t)f->B * f->L > (int64_t)INT32_MAX / 2)
+    return LSH_ERR_UNSUPPORTED;
+  return LSH_OK;
+}
+static bool ff_empty(const lsh_ff_problem* f) { return (int64_t)f->B * f->L == 0; }
+static bool all_aligned16(std::initializer_list<const void*> ps) {
+  for (const void* q : ps)
+    if (!aligned(q, 16)) return false;
+  return true;
+}
+// The reversible block's attention: bf16, head size 64, the same B, H, L.
+static lsh_status check_rev(const lsh_problem* p, const lsh_ff_problem* f) {
+  lsh_status st = check_problem(p);
+  if (st != LSH_OK) return st;
+  st = check_ff(f);
+  if (st != LSH_OK) return st;
+  if (p->B != f->B || p->H != f->H || p->L != f->L) return LSH_ERR_INVALID_ARG;
+  if (p->dtype != LSH_BF16) return LSH_ERR_UNSUPPORTED;
+  return LSH_OK;
+}
+
+size_t lsh_ff_workspace_size(const lsh_ff_problem* f) {
+  if (check_ff(f) != LSH_OK) return 0;
+  return ff_ws_bytes(*f);
+}
+
+lsh_status lsh_ff_fwd(const lsh_ff_problem* f, const void* x, const void* W1, const float* b1,
+                      const void* W2, const float* b2, const void* res, void* y, void* ws,
+                      size_t ws_bytes, lsh_stream_t stream) {
+  lsh_status st = check_ff(f);
+  if (st != LSH_OK) return st;
+  if (ff_empty(f)) return LSH_OK;
+  if (!x || !W1 || !b1 || !W2 || !b2 || !y) return LSH_ERR_INVALID_ARG;
+  if (!all_aligned16({x, W1, b1, W2, b2, res, y}) || x == y) return LSH_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < ff_ws_bytes(*f) || !aligned(ws, 256)) return LSH_ERR_WORKSPACE;
+  return cuda_status(launch_ff_fwd(*f, x, W1, b1, W2, b2, res, y, ws, device_status_word(),
+                                   (cudaStream_t)stream));
+}
+
+lsh_status lsh_ff_bwd(const lsh_ff_problem* f, const void* x, const void* W1, const float* b1,
+                      const void* W2, const float* b2, const void* dy, const void* dres,
+                      const void* y_in, void* rec, void* dx, float* dW1, float* db1, float* dW2,
+                      float* db2, void* ws, size_t ws_bytes, lsh_stream_t stream) {
+  lsh_status st = check_ff(f);
+  if (st != LSH_OK) return st;
+  if (ff_empty(f)) return LSH_OK;
+  if (!x || !W1 || !b1 || !W2 || !b2 || !dy || !dx || !dW1 || !db1 || !dW2 || !db2)
+    return LSH_ERR_INVALID_ARG;
+  if ((y_in == nullptr) != (rec == nullptr)) return LSH_ERR_INVALID_ARG;
+  if (!all_aligned16({x, W1, b1, W2, b2, dy, dres, y_in, rec, dx, dW1, db1, dW2, db2}))
+    return LSH_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < ff_ws_bytes(*f) || !aligned(ws, 256)) return LSH_ERR_WORKSPACE;
+  return cuda_status(launch_ff_bwd(*f, x, W1, b1, W2, b2, dy, dres, y_in, rec, dx, dW1, db1, dW2,
+                                   db2, ws, device_status_word(), (cudaStream_t)stream));
+}
+
+size_t lsh_rev_fwd_workspace_size(const lsh_problem* p, const lsh_ff_problem* f) {
+  if (check_rev(p, f) != LSH_OK) return 0;
+  return rev_fwd_ws_bytes(*p, *f);
+}
+
+lsh_status lsh_rev_fwd(const lsh_problem* p, const lsh_ff_problem* f, const void* x1,
+                       const void* x2, const void* R, const void* W1, const float* b1,
+                       const void* W2, const float* b2, void* y1, void* y2, int32_t* perm,
+                       void* ws, size_t ws_bytes, lsh_stream_t stream) {
+  lsh_status st = check_rev(p, f);
+  if (st != LSH_OK) return st;
+  if (empty(p)) return LSH_OK;
+  if (!x1 || !x2 || !R || !W1 || !b1 || !W2 || !b2 || !y1 || !y2 || !perm)
+    return LSH_ERR_INVALID_ARG;
+  if (!all_aligned16({x1, x2, R, W1, b1, W2, b2, y1, y2})) return LSH_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < rev_fwd_ws_bytes(*p, *f) || !aligned(ws, 256)) return LSH_ERR_WORKSPACE;
+  return cuda_status(launch_rev_fwd(*p, *f, x1, x2, R, W1, b1, W2, b2, y1, y2, perm, ws,
+                                    device_status_word(), (cudaStream_t)stream));
+}
+
+size_t lsh_rev_bwd_workspace_size(const lsh_problem* p, const lsh_ff_problem* f) {
+  if (check_rev(p, f) != LSH_OK) return 0;
+  return rev_bwd_ws_bytes(*p, *f);
+}
+
+lsh_status lsh_rev_bwd(const lsh_problem* p, const lsh_ff_problem* f, const void* y1,
+                       const void* y2, const void* dy1, const void* dy2, const int32_t* perm,
+                       const void* W1, const float* b1, const void* W2, const float* b2,
+                       void* x1, void* x2, void* dx1, void* dx2, float* dW1, float* db1,
+                       float* dW2, float* db2, void* ws, size_t ws_bytes, lsh_stream_t stream) {
+  lsh_status st = check_rev(p, f);
+  if (st != LSH_OK) return st;
+  if (empty(p)) return LSH_OK;
+  if (!y1 || !y2 || !dy1 || !dy2 || !perm || !W1 || !b1 || !W2 || !b2 || !x1 || !x2 || !dx1 ||
+      !dx2 || !dW1 || !db1 || !dW2 || !db2)
+    return LSH_ERR_INVALID_ARG;
+  if (!all_aligned16({y1, y2, dy1, dy2, W1, b1, W2, b2, x1, x2, dx1, dx2, dW1, db1, dW2, db2}))
+    return LSH_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < rev_bwd_ws_bytes(*p, *f) || !aligned(ws, 256)) return LSH_ERR_WORKSPACE;
+  return cuda_status(launch_rev_bwd(*p, *f, y1, y2, dy1, dy2, perm, W1, b1, W2, b2, x1, x2, dx1,
+                                    dx2, dW1, db1, dW2, db2, ws, device_status_word(),
+                                    (cudaStream_t)stream));
 }
 
 lsh_status lsh_device_status(lsh_stream_t stream) {

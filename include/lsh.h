@@ -177,6 +177,69 @@ lsh_status lsh_local_attn_bwd(const lsh_problem* p, int32_t n_back, int32_t n_fw
                               lsh_stream_t stream);
 
 /*
+ * The layer around the attention: a chunked position-wise feed-forward and
+ * the reversible residual block ("Reformer: The Efficient Transformer",
+ * research.elamur.ai summary page, Key points, "Reversible layers":
+ * reversible residual layers (Gomez et al. 2017) recompute a layer's inputs
+ * from its outputs in the backward pass instead of storing them; the
+ * feed-forward runs in chunks, which leaves its results unchanged).
+ *   G(x) = max(0, x W1 + b1) W2 + b2, applied to every position;
+ *   F(x2) = lsh_attn_fwd's output with qk = v = x2 (shared-QK attention whose
+ *           values are its input; projection weights are not part of this);
+ *   forward  y1 = x1 + F(x2), y2 = x2 + G(y1);
+ *   backward x2 = y2 - G(y1), x1 = y1 - F(x2), from the outputs alone.
+ * Activations x, x1, x2, y, y1, y2 and their gradients are [B, H, L, 64]
+ * bf16, the attention's layout: token (b, l) has d_model = 64 H features, its
+ * H head rows side by side. W1 [d_model, d_ff] and W2 [d_ff, d_model] are
+ * bf16 row-major; b1 [d_ff], b2 [d_model] and all weight gradients are
+ * float32. Products run on the tensor cores with float32 accumulation; the
+ * hidden activations and their gradient are rounded to bf16 per chunk.
+ * Every result is deterministic, and every per-position result (y, dx, the
+ * reconstruction) is bit-identical for any ff_chunk.
+ */
+typedef struct {
+  int32_t B, H, L;     /* activations [B, H, L, 64]; L a multiple of 128       */
+  int32_t d_ff;        /* hidden width: a multiple of 128, up to 65536         */
+  int32_t ff_chunk;    /* positions per feed-forward chunk: a multiple of 128 */
+} lsh_ff_problem;
+
+/* y = res + G(x) (res may be NULL: y = G(x)); y may not alias x. */
+size_t lsh_ff_workspace_size(const lsh_ff_problem* f);
+lsh_status lsh_ff_fwd(const lsh_ff_problem* f, const void* x, const void* W1, const float* b1,
+                      const void* W2, const float* b2, const void* res, void* y, void* ws,
+                      size_t ws_bytes, lsh_stream_t stream);
+/* Backward of y = res + G(x) for the incoming gradient dy:
+ *   dx = dres + (dG/dx)^T dy (dres may be NULL), bf16;
+ *   dW1, db1, dW2, db2 = gradients of sum(G(x) * dy), overwritten;
+ *   rec (optional): y_in - G(x), the reversible block's reconstruction of the
+ *   residual branch from its output y_in (both NULL, or both given).
+ * The workspace is that of lsh_ff_fwd. */
+lsh_status lsh_ff_bwd(const lsh_ff_problem* f, const void* x, const void* W1, const float* b1,
+                      const void* W2, const float* b2, const void* dy, const void* dres,
+                      const void* y_in, void* rec, void* dx, float* dW1, float* db1, float* dW2,
+                      float* db2, void* ws, size_t ws_bytes, lsh_stream_t stream);
+
+/* Reversible block forward: hashes x2 with R, sorts (perm, [B, H, n_rounds,
+ * L], is written for the backward), y1 = x1 + F(x2), y2 = x2 + G(y1).
+ * p describes the attention (bf16, d 64, same B, H, L as f). */
+size_t lsh_rev_fwd_workspace_size(const lsh_problem* p, const lsh_ff_problem* f);
+lsh_status lsh_rev_fwd(const lsh_problem* p, const lsh_ff_problem* f, const void* x1,
+                       const void* x2, const void* R, const void* W1, const float* b1,
+                       const void* W2, const float* b2, void* y1, void* y2, int32_t* perm,
+                       void* ws, size_t ws_bytes, lsh_stream_t stream);
+/* Reversible block backward from (y1, y2), the incoming gradients (dy1, dy2)
+ * and the forward's perm (kept, because a bucket id is a discrete function of
+ * x2 and the reconstruction recovers x2 only up to rounding): writes the
+ * reconstructed inputs x1, x2, their gradients dx1, dx2 (bf16) and the
+ * feed-forward's weight gradients (float32, overwritten). */
+size_t lsh_rev_bwd_workspace_size(const lsh_problem* p, const lsh_ff_problem* f);
+lsh_status lsh_rev_bwd(const lsh_problem* p, const lsh_ff_problem* f, const void* y1,
+                       const void* y2, const void* dy1, const void* dy2, const int32_t* perm,
+                       const void* W1, const float* b1, const void* W2, const float* b2,
+                       void* x1, void* x2, void* dx1, void* dx2, float* dW1, float* db1,
+                       float* dW2, float* db2, void* ws, size_t ws_bytes, lsh_stream_t stream);
+
+/*
  * lsh_sort_noalloc — lsh_sort without a caller workspace. The reference pages
  *   have no counterpart: this entry point exists for callers that cannot
  *   obtain device memory for a workspace, such as a host framework that owns

@@ -145,3 +145,65 @@ def test_local_attention_rejects_bad_arguments_before_launch():
     empty = _p(n_rounds=1, B=0)
     assert L.lsh_local_attn_fwd(ctypes.byref(empty), 1, 1, None, None, None, None, None, None, 0,
                                 None) == 0
+
+
+def _f(**kw):
+    base = dict(B=1, H=2, L=256, d_ff=256, ff_chunk=128)
+    base.update(kw)
+    return _lib.lsh_ff_problem(*[base[k] for k, _ in _lib.lsh_ff_problem._fields_])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(L=192), 1), (dict(d_ff=192), 1), (dict(d_ff=0), 1), (dict(ff_chunk=64), 1),
+    (dict(ff_chunk=200), 1), (dict(H=0), 1), (dict(B=-1), 1), (dict(d_ff=65536 + 128), 2),
+    (dict(H=1025), 2),
+])
+def test_feed_forward_rejects_bad_problem_before_launch(kw, code):
+    _ensure_built()
+    L = _lib.lib()
+    f = _f(**kw)
+    assert L.lsh_ff_workspace_size(ctypes.byref(f)) == 0
+    args = [FAKE] * 5 + [None, FAKE * 2, FAKE, 1 << 30, None]
+    assert L.lsh_ff_fwd(ctypes.byref(f), *args) == code
+
+
+def test_feed_forward_and_block_check_pointers_and_workspace():
+    _ensure_built()
+    L = _lib.lib()
+    f = _f()
+    n = L.lsh_ff_workspace_size(ctypes.byref(f))
+    assert n > 0 and n % 256 == 0
+    ok = [FAKE] * 5 + [None, FAKE * 2]
+    assert L.lsh_ff_fwd(ctypes.byref(f), *ok, FAKE, n - 1, None) == 3
+    assert L.lsh_ff_fwd(ctypes.byref(f), *ok, None, n, None) == 3
+    assert L.lsh_ff_fwd(ctypes.byref(f), None, *ok[1:], FAKE, n, None) == 1
+    assert L.lsh_ff_fwd(ctypes.byref(f), FAKE, *ok[1:6], FAKE, FAKE, n, None) == 1   # y aliases x
+    assert L.lsh_ff_fwd(ctypes.byref(f), FAKE + 8, *ok[1:], FAKE, n, None) == 1      # misaligned x
+    bwd = [FAKE] * 6 + [None, None, None] + [FAKE] * 5
+    assert L.lsh_ff_bwd(ctypes.byref(f), *bwd, FAKE, n - 1, None) == 3
+    bad = list(bwd)
+    bad[7] = FAKE                      # y_in without rec
+    assert L.lsh_ff_bwd(ctypes.byref(f), *bad, FAKE, n, None) == 1
+    p = _p(n_rounds=2)
+    assert L.lsh_rev_fwd_workspace_size(ctypes.byref(p), ctypes.byref(f)) > 0
+    assert L.lsh_rev_bwd_workspace_size(ctypes.byref(p), ctypes.byref(f)) > 0
+    # the attention must match the block's B, H, L and be bf16
+    for pk in (dict(H=3), dict(L=512), dict(dtype=0)):
+        q = _p(**pk)
+        assert L.lsh_rev_fwd_workspace_size(ctypes.byref(q), ctypes.byref(f)) == 0
+        assert L.lsh_rev_fwd(ctypes.byref(q), ctypes.byref(f), *([FAKE] * 10), FAKE, 1 << 30,
+                             None) in (1, 2)
+    nr = L.lsh_rev_bwd_workspace_size(ctypes.byref(p), ctypes.byref(f))
+    assert L.lsh_rev_bwd(ctypes.byref(p), ctypes.byref(f), *([FAKE] * 17), FAKE, nr - 1,
+                         None) == 3
+
+
+def test_feed_forward_and_block_empty_problem_is_a_noop():
+    _ensure_built()
+    L = _lib.lib()
+    f = _f(B=0)
+    assert L.lsh_ff_fwd(ctypes.byref(f), *([None] * 8), 0, None) == 0
+    assert L.lsh_ff_bwd(ctypes.byref(f), *([None] * 15), 0, None) == 0
+    p = _p(B=0)
+    assert L.lsh_rev_fwd(ctypes.byref(p), ctypes.byref(f), *([None] * 11), 0, None) == 0
+    assert L.lsh_rev_bwd(ctypes.byref(p), ctypes.byref(f), *([None] * 18), 0, None) == 0
