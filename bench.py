@@ -25,8 +25,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from efficient_transformer_lsh_b200.workloads import (HEADLINE, WORKLOADS, generate,  # noqa: E402
-                                                      generate_slices)
+from efficient_transformer_lsh_b200.workloads import (BLOCK_FF, HEADLINE, WORKLOADS,  # noqa: E402
+                                                      generate, generate_block, generate_slices)
 
 METRIC = "LSH-attn fwd+bwd tokens/s at L=64K, 8 heads, 4 rounds; % of roofline"
 UNIT = "tokens/s"
@@ -59,6 +59,88 @@ def stage_models(w):
         "fwd": {"bytes": fwd_b, "flops": attn_fwd_flops},
         "bwd": {"bytes": bwd_b if w.backward else 0,
                 "flops": 2.5 * attn_fwd_flops if w.backward else 0},
+    }
+
+
+def bench_block(w, dev, stream, steps, warmup, peaks):
+    """One Reformer layer around this workload's attention: the reversible
+    block forward (hash, sort, y1 = x1 + F(x2), y2 = x2 + G(y1)) and backward
+    (x2 = y2 - G(y1), x1 = y1 - F(x2), all gradients), timed with CUDA events
+    on `stream`; then the chunked feed-forward alone (lsh_ff_fwd, and
+    lsh_ff_bwd with the reconstruction) against the tensor-core peak.
+    Every step touches well over the L2's 126 MB (ten 64 MB activations)."""
+    import torch
+
+    from efficient_transformer_lsh_b200 import _lib
+    from efficient_transformer_lsh_b200.attention import ReversibleLSHBlock
+
+    cfg = BLOCK_FF[w.name]
+    d_ff, ff_chunk = cfg["d_ff"], cfg["ff_chunk"]
+    inp = generate_block(w, d_ff)
+    t = {k: torch.from_numpy(a).to(dev).to(torch.float32 if k in ("b1", "b2") else torch.bfloat16)
+         for k, a in inp.items()}
+    blk = ReversibleLSHBlock(w.B, w.H, w.L, w.n_buckets, w.n_rounds, w.chunk, w.causal, d_ff,
+                             ff_chunk, w.scale, dev)
+    W = (t["W1"], t["b1"], t["W2"], t["b2"])
+
+    def fwd():
+        blk.forward(t["x1"], t["x2"], t["R"], *W, stream)
+
+    def bwd():
+        blk.backward(blk.y1, blk.y2, t["dy1"], t["dy2"], *W, stream)
+
+    f = blk.f
+    nff = _lib.lsh_ff_workspace_size(f)
+    wsff = torch.empty(nff, dtype=torch.uint8, device=dev)
+    y, rec, dx = (torch.empty_like(t["x1"]) for _ in range(3))
+    g = (blk.dW1, blk.db1, blk.dW2, blk.db2)
+
+    def ff_fwd():
+        _lib.lsh_ff_fwd(f, t["x1"], *W, t["x2"], y, wsff, nff, stream)
+
+    def ff_bwd():
+        _lib.lsh_ff_bwd(f, t["x1"], *W, t["dy2"], t["dy1"], y, rec, dx, *g, wsff, nff, stream)
+
+    def timed(fns):
+        for _ in range(warmup):
+            for fn in fns:
+                fn()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+               for _ in range(steps)]
+        torch.cuda.synchronize(dev)
+        for k in range(steps):
+            for i, fn in enumerate(fns):
+                evs[k][i].record(stream)
+                fn()
+            evs[k][-1].record(stream)
+        torch.cuda.synchronize(dev)
+        return [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(steps))
+                for i in range(len(fns))]
+
+    launches0 = _lib.lsh_launch_count()
+    ms_fwd, ms_bwd = timed([fwd, bwd])
+    ff_ms_fwd, ff_ms_bwd = timed([ff_fwd, ff_bwd])
+    launches = (_lib.lsh_launch_count() - launches0) // (2 * (warmup + steps))
+    assert _lib.lsh_device_status(stream) == 0
+    T, D = w.B * w.L, w.H * w.d
+    gemm = 2.0 * T * D * d_ff            # FLOPs of one feed-forward product
+    tf_fwd = 2 * gemm / (ff_ms_fwd / 1e3) / 1e12
+    tf_bwd = 6 * gemm / (ff_ms_bwd / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
+    return {
+        "what": "reversible block y1 = x1 + LSHAttn(x2), y2 = x2 + FF(y1), forward + backward "
+                "from the outputs; the feed-forward alone below",
+        "d_model": D, "d_ff": d_ff, "ff_chunk": ff_chunk, "steps": steps,
+        "ms_fwd": ms_fwd, "ms_bwd": ms_bwd, "ms_per_step": ms_fwd + ms_bwd,
+        "tokens_per_s": T / ((ms_fwd + ms_bwd) / 1e3),
+        "launches_per_step": launches,
+        "ff": {"ms_fwd": ff_ms_fwd, "ms_bwd": ff_ms_bwd,
+               "flops_fwd": 2 * gemm, "flops_bwd": 6 * gemm,
+               "tflops_fwd": tf_fwd, "tflops_bwd": tf_bwd, "peak_tflops": peak,
+               "frac_fwd": tf_fwd / peak, "frac_bwd": tf_bwd / peak,
+               "peak_source": peaks["source"],
+               "note": "fwd: h = relu(x W1 + b1), y = res + h W2 + b2; bwd: h again, "
+                       "the reconstruction, dh, dW2, dW1, dx (six products)"},
     }
 
 
@@ -277,6 +359,8 @@ def main():
     ap.add_argument("--heads", type=int, default=None,
                     help="override H (smaller cases of the same kernels, e.g. for profiler captures)")
     ap.add_argument("--seq-len", type=int, default=None, help="override L")
+    ap.add_argument("--no-block", action="store_true",
+                    help="skip the reversible-block (attention + chunked feed-forward) timing")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     if args.heads is not None:
@@ -476,6 +560,9 @@ def main():
         "e2e": e2e, "gpu_launches": launches, "clocks": sampler.summary(t_host0, t_host1),
         "memory": memory,
     }
+    if rank == 0 and world == 1 and not args.no_block and w.name in BLOCK_FF and \
+            args.heads is None and args.seq_len is None:
+        line["rev_block"] = bench_block(w, dev, stream, min(K, 10), args.warmup, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:

@@ -12,8 +12,10 @@
 // matrix or from the attention's [B, H, L, 64] activation layout, in which
 // token row (b, l) has its 64 H features spread over the H head rows.
 //
-// One CTA computes one 128 x BN tile (BN = 64 or 128), K in steps of 64:
-//   warp 0     : one lane issues the TMA loads into a 4-stage ring;
+// One CTA computes one 128 x BN tile (BN = 64 or 128), K in steps of 64; two
+// CTAs fit on an SM (97 KB of shared memory each), so one's epilogue runs
+// under the other's main loop:
+//   warp 0     : one lane issues the TMA loads into a 3-stage ring;
 //   warp 1     : TMEM allocation; one lane issues the MMAs (128 x BN x 16);
 //   warps 2-5  : epilogue, one thread per tile row (TMEM lane): bias, ReLU,
 //                mask, residual, then bf16 or fp32 stores (optionally
@@ -34,7 +36,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kBM = 128, kBK = 64, kStages = 4;
+constexpr int kBM = 128, kBK = 64, kStages = 3;
 constexpr int kThreads = 192;
 constexpr int kATile = kBM * kBK * 2;   // 16 KB
 
@@ -64,7 +66,7 @@ __device__ __forceinline__ void load_box(void* dst, const CUtensorMap* map, int 
 }
 
 template <int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                GemmOpDev a, GemmOpDev b, int K, GemmEpi e, int* status) {
   extern __shared__ uint8_t smem_raw[];

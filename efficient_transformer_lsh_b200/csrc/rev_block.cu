@@ -71,19 +71,26 @@ sum3_kernel(const __nv_bfloat16* __restrict__ a, const float* __restrict__ g1,
   reinterpret_cast<uint4*>(out)[k] = make_uint4(r[0], r[1], r[2], r[3]);
 }
 
-// db[c] (+)= sum over rows r0 .. r0+rows-1 of src(row, c), c < N. src is a
-// plain [*, ld] bf16 matrix or the head layout (token rows, 64 H columns).
-// Thread (x, y) of a 32 x 8 block sums the rows y, y+8, ... of column
-// 32 blockIdx.x + x in order; the 8 partial sums are then added in y order,
-// so the result does not depend on scheduling.
+// Column sums of a bf16 block, in two deterministic passes.
+// src(row, c) is a plain [*, ld] matrix or the head layout (token rows, 64 H
+// columns, row g = b L + l). Pass 1: block (x, y) takes 256 columns and the
+// kSumRows rows starting at y kSumRows; warp w of it adds rows w, w + 8, ...
+// (16-byte loads, 8 columns a thread), then the 8 warps' sums are added in
+// warp order into part[y][c]. Pass 2: db[c] (+)= the parts in y order.
+constexpr int kSumRows = 256;
+
 __global__ void __launch_bounds__(256)
-colsum_kernel(const __nv_bfloat16* __restrict__ src, int heads, int64_t r0, int rows, int N,
-              int64_t ld, int L, int H, float* __restrict__ db, int accumulate) {
-  __shared__ float part[8][32];
-  const int c = blockIdx.x * 32 + threadIdx.x;
-  float s = 0.f;
+colsum_part_kernel(const __nv_bfloat16* __restrict__ src, int heads, int64_t r0, int rows, int N,
+                   int64_t ld, int L, int H, float* __restrict__ part) {
+  __shared__ float red[8][256];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int c = blockIdx.x * 256 + lane * 8;
+  const int lo = blockIdx.y * kSumRows, hi = min(rows, lo + kSumRows);
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
   if (c < N) {
-    for (int r = threadIdx.y; r < rows; r += 8) {
+    for (int r = lo + w; r < hi; r += 8) {
       const int64_t g = r0 + r;
       int64_t off;
       if (heads) {
@@ -92,24 +99,45 @@ colsum_kernel(const __nv_bfloat16* __restrict__ src, int heads, int64_t r0, int 
       } else {
         off = g * ld + c;
       }
-      s += __bfloat162float(src[off]);
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + off));
+      const uint32_t v[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] += bf_lo(v[i]);
+        acc[2 * i + 1] += bf_hi(v[i]);
+      }
     }
   }
-  part[threadIdx.y][threadIdx.x] = s;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) red[w][lane * 8 + i] = acc[i];
   __syncthreads();
-  if (threadIdx.y == 0 && c < N) {
+  const int cc = blockIdx.x * 256 + threadIdx.x;
+  if (cc < N) {
     float t = 0.f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) t += part[k][threadIdx.x];
-    db[c] = accumulate ? db[c] + t : t;
+    for (int k = 0; k < 8; ++k) t += red[k][threadIdx.x];
+    part[(int64_t)blockIdx.y * N + cc] = t;
   }
 }
 
+__global__ void __launch_bounds__(256)
+colsum_final_kernel(const float* __restrict__ part, int S, int N, float* __restrict__ db,
+                    int accumulate) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= N) return;
+  float t = 0.f;
+  for (int k = 0; k < S; ++k) t += part[(int64_t)k * N + c];
+  db[c] = accumulate ? db[c] + t : t;
+}
+
 cudaError_t colsum(const __nv_bfloat16* src, int heads, int64_t r0, int rows, int N, int64_t ld,
-                   int L, int H, float* db, bool accumulate, cudaStream_t s) {
-  colsum_kernel<<<(unsigned)((N + 31) / 32), dim3(32, 8), 0, s>>>(src, heads, r0, rows, N, ld, L, H,
-                                                                 db, accumulate ? 1 : 0);
-  note_launch();
+                   int L, int H, float* part, float* db, bool accumulate, cudaStream_t s) {
+  const int S = (rows + kSumRows - 1) / kSumRows;
+  colsum_part_kernel<<<dim3((unsigned)((N + 255) / 256), (unsigned)S), 256, 0, s>>>(
+      src, heads, r0, rows, N, ld, L, H, part);
+  colsum_final_kernel<<<(unsigned)((N + 255) / 256), 256, 0, s>>>(part, S, N, db,
+                                                                  accumulate ? 1 : 0);
+  note_launch(2);
   return cudaGetLastError();
 }
 
@@ -142,11 +170,18 @@ GemmEpi epi() {
 struct FfWs {
   __nv_bfloat16* h;    // [ff_chunk, d_ff] hidden block
   __nv_bfloat16* dh;   // [ff_chunk, d_ff] its gradient
+  float* part;         // partial column sums of the bias gradients
 };
+size_t ff_part_bytes(const lsh_ff_problem& f) {
+  const size_t S = ((size_t)f.ff_chunk + kSumRows - 1) / kSumRows;
+  return align_up(S * (size_t)std::max(f.d_ff, 64 * f.H) * 4, 256);
+}
 FfWs ff_carve(const lsh_ff_problem& f, void* ws) {
   FfWs w;
+  const size_t hb = align_up((size_t)f.ff_chunk * f.d_ff * 2, 256);
   w.h = (__nv_bfloat16*)ws;
-  w.dh = (__nv_bfloat16*)((char*)ws + align_up((size_t)f.ff_chunk * f.d_ff * 2, 256));
+  w.dh = (__nv_bfloat16*)((char*)ws + hb);
+  w.part = (float*)((char*)ws + 2 * hb);
   return w;
 }
 
@@ -186,7 +221,7 @@ cudaError_t ff_out(const lsh_ff_problem& f, const __nv_bfloat16* h, const void* 
 }  // namespace
 
 size_t ff_ws_bytes(const lsh_ff_problem& f) {
-  return 2 * align_up((size_t)f.ff_chunk * f.d_ff * 2, 256);
+  return 2 * align_up((size_t)f.ff_chunk * f.d_ff * 2, 256) + ff_part_bytes(f);
 }
 
 cudaError_t launch_ff_fwd(const lsh_ff_problem& f, const void* x, const void* W1, const float* b1,
@@ -271,9 +306,9 @@ cudaError_t launch_ff_bwd(const lsh_ff_problem& f, const void* x, const void* W1
                          ep, status, s);
       if (e != cudaSuccess) return e;
     }
-    e = colsum(w.dh, 0, 0, Mc, f.d_ff, f.d_ff, f.L, f.H, db1, acc, s);
+    e = colsum(w.dh, 0, 0, Mc, f.d_ff, f.d_ff, f.L, f.H, w.part, db1, acc, s);
     if (e != cudaSuccess) return e;
-    e = colsum((const __nv_bfloat16*)dy, 1, r0, Mc, D, 0, f.L, f.H, db2, acc, s);
+    e = colsum((const __nv_bfloat16*)dy, 1, r0, Mc, D, 0, f.L, f.H, w.part, db2, acc, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -114,6 +114,7 @@ def _to_dtype(a: np.ndarray, dtype: str) -> np.ndarray:
 
 
 _QK, _V, _DO, _R, _CENTRES = 0, 1, 2, 3, 4
+_W1, _B1, _W2, _B2, _DY1 = 5, 6, 7, 8, 9
 
 
 def _stream(seed: int, array: int, k: int = 0) -> np.random.Generator:
@@ -166,4 +167,30 @@ def generate(w: Workload, seed: Optional[int] = None, with_grad: Optional[bool] 
     for k in ("qk", "v", "dO"):
         if k in out:
             out[k] = out[k].reshape(w.B, w.H, w.L, w.d)
+    return out
+
+
+# The reversible block around the attention (one Reformer layer) on a workload:
+# d_model = 64 H, a feed-forward of width 4 d_model run ff_chunk positions at a
+# time.
+BLOCK_FF = {"enwik8-64k-bf16": dict(d_ff=2048, ff_chunk=8192)}
+
+
+def generate_block(w: Workload, d_ff: int, seed: Optional[int] = None):
+    """Inputs of the reversible block on workload ``w`` (bf16): x2 = the
+    workload's qk (so the hash sees its bucket structure), x1 = its v,
+    dy2 = its dO, dy1 ~ N(0, 1), all [B, H, L, d]; R as drawn; W1 [64 H, d_ff]
+    ~ N(0, 1/(64 H)), W2 [d_ff, 64 H] ~ N(0, 1/d_ff) (bf16) and b1, b2 ~
+    N(0, 0.1^2) (float32)."""
+    if seed is None:
+        seed = 20200 + w.index
+    base = generate(w, seed, with_grad=True)
+    D = w.H * w.d
+    out = {"x1": base["v"], "x2": base["qk"], "R": base["R"], "dy2": base["dO"]}
+    out["dy1"] = round_to_bf16(np.stack([_stream(seed, _DY1, k).standard_normal((w.L, w.d))
+                                         for k in range(w.B * w.H)])).reshape(w.B, w.H, w.L, w.d)
+    out["W1"] = round_to_bf16(_stream(seed, _W1).standard_normal((D, d_ff)) / np.sqrt(D))
+    out["W2"] = round_to_bf16(_stream(seed, _W2).standard_normal((d_ff, D)) / np.sqrt(d_ff))
+    out["b1"] = (0.1 * _stream(seed, _B1).standard_normal(d_ff)).astype(np.float32)
+    out["b2"] = (0.1 * _stream(seed, _B2).standard_normal(D)).astype(np.float32)
     return out
