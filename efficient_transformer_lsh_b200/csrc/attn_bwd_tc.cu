@@ -27,9 +27,9 @@
 //        so that the next item of the same unit adds its own terms on top.
 //        At the end of a unit it is stored on its own (the edge rows below).
 // The finished rows dV and scale*dK of an item are stored, converted to fp16,
-// as per-round partial gradients in token order: each flush thread writes its
-// key row's two 128-byte rows at the row's position, so every round's
-// partial is a plain (position, 64) array. Unit-end R1 rows go to a small
+// as per-round partial gradients in token order: each key row's two 128-byte
+// rows go to the row's position, so every round's partial is a plain
+// (position, 64) array. Unit-end R1 rows go to a small
 // edge buffer, and the first item of the next unit records, per position of
 // its first chunk, which edge row belongs to it (-1 for every other
 // position). A second kernel then streams the rounds' partials of every
@@ -48,8 +48,9 @@
 //   warp 3     : TMEM allocation and the MMA issue (the warp waits
 //                converged; one elected lane issues each MMA and commit);
 //   warps 4-7  : gradient flush of the previous item (one thread per key
-//                row: TMEM -> fp16 -> a padded staging row -> one bulk copy
-//                to the row's place in the partial arrays);
+//                row: TMEM -> fp16 -> a padded staging row; then each warp
+//                stores its 32 rows, four whole rows per store instruction,
+//                at their places in the partial arrays);
 //   warps 8-23 : four softmax warpgroups, two per S^T buffer (even and odd
 //                steps), one thread per key row and 32 of the block's 64
 //                query columns each.
@@ -157,13 +158,15 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 // one lane never leaves the others inside a warp-collective instruction.
 __device__ __forceinline__ bool warp_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
 
-// Converts 64 fp32 TMEM columns of this thread's lane, times `sc`, to fp16,
-// places them in this thread's row of the staging area (rows 144 bytes apart,
-// so the 16-byte stores of eight consecutive rows fall in different banks)
-// and copies the 128 bytes to the global row `dst` with one bulk copy. The
-// staging row is free again when the function returns.
-__device__ __forceinline__ void put_row(uint32_t ta, float sc, uint8_t* srow, __half* dst,
-                                        bool live) {
+// Converts 64 fp32 TMEM columns of this thread's lane, times `sc`, to fp16
+// into the thread's row of its warp's 32 staging rows (144 bytes apart, so the
+// 16-byte stores of eight consecutive rows fall in different banks); then the
+// warp copies the 32 rows out, four whole 128-byte rows per store instruction
+// (eight lanes of 16 bytes each): row k goes to base + lane k's `off`
+// (halves), unless lane k's `live` is false.
+__device__ __forceinline__ void put_rows(uint32_t ta, float sc, uint8_t* wstage, int lane,
+                                         __half* base, int64_t off, bool live) {
+  uint8_t* srow = wstage + lane * kStageRow;
 #pragma unroll
   for (int h = 0; h < 4; ++h) {
     uint32_t a[16];
@@ -177,10 +180,19 @@ __device__ __forceinline__ void put_row(uint32_t ta, float sc, uint8_t* srow, __
     d[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     d[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
   }
-  fence_proxy_async();
-  if (live) bulk_store(dst, smem_u32(srow), 128);
-  bulk_commit();
-  bulk_wait_read_all();
+  __syncwarp();
+  const int sub = lane >> 3, ch = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int k = 4 * i + sub;
+    const long long ok = __shfl_sync(0xffffffffu, (long long)off, k);
+    const int lk = __shfl_sync(0xffffffffu, live ? 1 : 0, k);
+    if (lk) {
+      const uint4 v = *reinterpret_cast<const uint4*>(wstage + k * kStageRow + ch * 16);
+      *reinterpret_cast<uint4*>(base + ok + ch * 8) = v;
+    }
+  }
+  __syncwarp();
 }
 
 // ---- MMA issue helpers (one thread). Descriptor lower words: `sl` is the
@@ -464,7 +476,7 @@ attn_bwd_tc_kernel(const __half* __restrict__ qk, const __half* __restrict__ v,
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
-    uint8_t* srow = stage + row * kStageRow;
+    uint8_t* wstage = stage + q * 32 * kStageRow;
     JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
     Job j;
     int n = 0;
@@ -479,19 +491,18 @@ attn_bwd_tc_kernel(const __half* __restrict__ qk, const __half* __restrict__ v,
       const uint32_t acc = tl + kColAcc + (uint32_t)a * 128;
       const bool r1 = j.last && nc == 3;
       const int unit = (int)(j.seg * units_per_seg + j.p / kUnit);
-      put_row(acc, 1.f, srow, part_dv + rr * 64, live);
-      put_row(acc + 64, scale, srow, part_dqk + rr * 64, live);
+      put_rows(acc, 1.f, wstage, lane, part_dv, rr * 64, live);
+      put_rows(acc + 64, scale, wstage, lane, part_dqk, rr * 64, live);
       // the rows of a unit's first chunk (after the first unit) take the R1
       // rows that the previous unit's last item stored on its own
       if (live) emap[rr] = (j.first && j.p > 0 && row < kM) ? (unit - 1) * kM + row : -1;
       if (r1 && q < 2)
-        put_row(tl + kColAcc + (uint32_t)(a ^ 1) * 128 + 64, scale, srow,
-                edge + ((int64_t)unit * kM + row) * 64, true);
+        put_rows(tl + kColAcc + (uint32_t)(a ^ 1) * 128 + 64, scale, wstage, lane, edge,
+                 ((int64_t)unit * kM + row) * 64, true);
       tc_fence_before();
       mbar_arrive(&bar->acc_free[a]);
       ++n;
     }
-    bulk_wait_all();
   } else {
     // ------------------------------------------------ softmax: P^T and dS^T
     // Two warpgroups per S^T buffer, each owning 32 of the block's 64 query
