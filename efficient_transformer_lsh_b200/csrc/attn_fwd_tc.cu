@@ -27,9 +27,11 @@
 //                O = P V with P read from TMEM (A operand) and V from shared
 //                memory (MN-major B operand);
 //   warps 4-7  : softmax warpgroup for even jobs, warps 8-11 for odd jobs —
-//                one query row per thread, two passes over its S row in TMEM:
-//                (1) causal/self mask and row max, masked values written back;
-//                (2) exp2, row sum, P packed as fp16 pairs into TMEM over S.
+//                one query row per thread, two passes over its 128 scores,
+//                held in registers (the second 64-column TMEM load in flight
+//                while the first block is masked): (1) causal/self mask and
+//                row max; (2) exp2, row sum, P packed as fp16 pairs into TMEM
+//                over S.
 //                After publishing P, the warpgroup writes its previous job's
 //                output: O from TMEM scaled by 1/l, as fp16, in original token
 //                order, + lse_r (so the stores stay off the path from S to P).
@@ -436,13 +438,20 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __half* __restric
       // (-inf) are written back so pass 2 needs no positions. Two TMEM loads
       // per wait and four independent max chains keep latency off the path.
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // the second 64-column block's TMEM load is in flight while the first
+      // one is masked (and, in pass 2, exponentiated)
+      uint32_t sv[2][64];
+      const uint32_t col0 = (uint32_t)(kb0 * 64), col1 = col0 + 64;
+      tmem_ld32(sbuf + col0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0][0]));
+      tmem_ld32(sbuf + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[0][32]));
+      tmem_ld_wait();
 #pragma unroll
       for (int c2 = 0; c2 < 2; ++c2) {
-        const uint32_t col = (uint32_t)(kb0 * 64 + c2 * 64);
-        uint32_t sv[64];
-        tmem_ld32(sbuf + col, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(sbuf + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld_wait();
+        if (c2 == 0) {
+          tmem_ld32(sbuf + col1, *reinterpret_cast<uint32_t(*)[32]>(&sv[1][0]));
+          tmem_ld32(sbuf + col1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[1][32]));
+        }
+        const uint32_t col = c2 ? col1 : col0;
         const int* kp = (c2 == 0) ? kp_lo : kp_hi;
         const bool blk_ok = (c2 == 0) ? lo_ok : true;
 #pragma unroll
@@ -454,33 +463,28 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __half* __restric
           for (int e = 0; e < 4; ++e) {
             const int i = 4 * i4 + e;
             const bool valid = blk_ok && (kCausal ? (kk[e] < qpos) : (kk[e] != qpos));
-            const float x = valid ? __uint_as_float(sv[i]) : -INFINITY;
-            sv[i] = __float_as_uint(x);
+            const float x = valid ? __uint_as_float(sv[c2][i]) : -INFINITY;
+            sv[c2][i] = __float_as_uint(x);
             mx4[e] = fmaxf(mx4[e], x);
           }
         }
-        tmem_st32(sbuf + col, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_st32(sbuf + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        (void)col;
+        if (c2 == 0) tmem_ld_wait();
       }
-      tmem_st_wait();
       const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       const bool has = mx != -INFINITY;
       const float neg = has ? -mx * scale_log2 : 0.f;
       // pass 2: P = exp2(scale * (s - max)) as fp16 pairs into TMEM over S;
-      // P column block kb lives at TMEM columns [32 kb, 32 kb + 32)
+      // P column block kb lives at TMEM columns [32 kb, 32 kb + 32). The masked
+      // values are still in registers, so nothing is read back.
       float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c2 = 0; c2 < 2; ++c2) {
-        uint32_t sv[64];
-        const uint32_t col = (uint32_t)(kb0 * 64 + c2 * 64);
-        tmem_ld32(sbuf + col, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(sbuf + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld_wait();
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float e0 = ex2(fmaf(__uint_as_float(sv[2 * e]), scale_log2, neg));
-          const float e1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), scale_log2, neg));
+          const float e0 = ex2(fmaf(__uint_as_float(sv[c2][2 * e]), scale_log2, neg));
+          const float e1 = ex2(fmaf(__uint_as_float(sv[c2][2 * e + 1]), scale_log2, neg));
           l4[e & 3] += e0 + e1;
           pk[e] = pack_f16x2(e0, e1);
         }

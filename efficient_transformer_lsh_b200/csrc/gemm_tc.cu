@@ -39,6 +39,7 @@ using namespace tc;
 constexpr int kBM = 128, kBK = 64, kStages = 3;
 constexpr int kThreads = 192;
 constexpr int kATile = kBM * kBK * 2;   // 16 KB
+constexpr int kMaxSplits = kGemmMaxSplits;
 
 struct __align__(8) GemmBar {
   uint64_t full[kStages];
@@ -78,7 +79,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
   volatile int* abort = &bar->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * BN;
-  const int nk = K / kBK;
+  // K blocks [kb0, kb0 + nk) of this CTA (gridDim.z splits of K)
+  const int nk = K / kBK / (int)gridDim.z;
+  const int kb0 = (int)blockIdx.z * nk;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -112,19 +115,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         uint8_t* da = sa + s * kATile;
         uint8_t* db = sb + s * kBTile;
         if (a.mn_major) {
-          load_box(da, &map_a, a.heads, a.L, a.row0 + (int64_t)kb * kBK, m0 / 64, &bar->full[s]);
-          load_box(da + kATile / 2, &map_a, a.heads, a.L, a.row0 + (int64_t)kb * kBK, m0 / 64 + 1,
+          load_box(da, &map_a, a.heads, a.L, a.row0 + (int64_t)(kb0 + kb) * kBK, m0 / 64,
                    &bar->full[s]);
+          load_box(da + kATile / 2, &map_a, a.heads, a.L, a.row0 + (int64_t)(kb0 + kb) * kBK,
+                   m0 / 64 + 1, &bar->full[s]);
         } else {
-          load_box(da, &map_a, a.heads, a.L, a.row0 + m0, kb, &bar->full[s]);
+          load_box(da, &map_a, a.heads, a.L, a.row0 + m0, kb0 + kb, &bar->full[s]);
         }
         if (b.mn_major) {
 #pragma unroll
           for (int i = 0; i < BN / 64; ++i)
             load_box(db + i * (64 * 128), &map_b, b.heads, b.L,
-                     b.row0 + (int64_t)kb * kBK, n0 / 64 + i, &bar->full[s]);
+                     b.row0 + (int64_t)(kb0 + kb) * kBK, n0 / 64 + i, &bar->full[s]);
         } else {
-          load_box(db, &map_b, b.heads, b.L, b.row0 + n0, kb, &bar->full[s]);
+          load_box(db, &map_b, b.heads, b.L, b.row0 + n0, kb0 + kb, &bar->full[s]);
         }
       }
     }
@@ -180,6 +184,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         float v[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(acc[i]);
+        if (e.split_part) {
+          // one K split's raw sums; split_reduce_kernel adds the splits
+          float4* op = reinterpret_cast<float4*>(
+              e.split_part + ((int64_t)blockIdx.z * e.M + row) * e.ldo + c);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            op[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          continue;
+        }
         if (e.bias) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] += __ldg(e.bias + c + i);
@@ -252,6 +265,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
   }
 }
 
+// out (+)= the S splits' partial sums, added in split order (float4 units).
+__global__ void __launch_bounds__(256)
+split_reduce_kernel(const float* __restrict__ part, int S, int64_t n4, float* __restrict__ out,
+                    int accumulate) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  float4 a = accumulate ? reinterpret_cast<const float4*>(out)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int z = 0; z < S; ++z) {
+    const float4 p = __ldg(reinterpret_cast<const float4*>(part) + z * n4 + i);
+    a.x += p.x;
+    a.y += p.y;
+    a.z += p.z;
+    a.w += p.w;
+  }
+  reinterpret_cast<float4*>(out)[i] = a;
+}
+
 // Tensor map of one operand: plain (cols, rows, 1, 1) or head layout
 // (64, L, H, B); box of 64 inner elements by `box_rows` rows.
 bool encode_op(CUtensorMap* map, const GemmOpHost& o, uint32_t box_rows) {
@@ -278,7 +308,7 @@ bool encode_op(CUtensorMap* map, const GemmOpHost& o, uint32_t box_rows) {
 }
 
 template <int BN>
-cudaError_t launch_bn(const GemmOpHost& a, const GemmOpHost& b, int M, int N, int K,
+cudaError_t launch_bn(const GemmOpHost& a, const GemmOpHost& b, int M, int N, int K, int splits,
                       const GemmEpi& e, int* status, cudaStream_t s) {
   CUtensorMap ma, mb;
   if (!encode_op(&ma, a, a.mn_major ? 64 : kBM) || !encode_op(&mb, b, b.mn_major ? 64 : BN))
@@ -289,9 +319,15 @@ cudaError_t launch_bn(const GemmOpHost& a, const GemmOpHost& b, int M, int N, in
   cudaError_t err =
       cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  const dim3 grid((unsigned)((M + kBM - 1) / kBM), (unsigned)(N / BN));
+  const dim3 grid((unsigned)((M + kBM - 1) / kBM), (unsigned)(N / BN), (unsigned)splits);
   gemm_tc_kernel<BN><<<grid, kThreads, smem, s>>>(ma, mb, da, db, K, e, status);
   note_launch();
+  if (e.split_part) {
+    const int64_t n4 = (int64_t)M * N / 4;
+    split_reduce_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(
+        e.split_part, splits, n4, (float*)e.out, e.accumulate);
+    note_launch();
+  }
   return cudaGetLastError();
 }
 
@@ -300,8 +336,24 @@ cudaError_t launch_bn(const GemmOpHost& a, const GemmOpHost& b, int M, int N, in
 cudaError_t launch_gemm_tc(const GemmOpHost& a, const GemmOpHost& b, int M, int N, int K,
                            const GemmEpi& e, int* status, cudaStream_t s) {
   if (M <= 0 || N <= 0 || K <= 0 || K % kBK != 0 || N % 64 != 0) return cudaErrorInvalidValue;
-  if (N % 128 == 0) return launch_bn<128>(a, b, M, N, K, e, status, s);
-  return launch_bn<64>(a, b, M, N, K, e, status, s);
+  const int bn = N % 128 == 0 ? 128 : 64;
+  int splits = 1;
+  if (e.split_part) {
+    // a plain float32 product (no epilogue terms) with few tiles: split K
+    // so that about one CTA per SM runs, in pieces of at least 4 K blocks
+    if (!e.out_f32 || e.out_heads || e.bias || e.relu || e.mask || e.res || e.ldo != N ||
+        e.row0 != 0)
+      return cudaErrorInvalidValue;
+    const int tiles = ((M + kBM - 1) / kBM) * (N / bn);
+    const int nk = K / kBK;
+    while (splits < kMaxSplits && tiles * splits * 2 <= sm_count() && nk % (splits * 2) == 0 &&
+           nk / (splits * 2) >= 4)
+      splits *= 2;
+  }
+  GemmEpi e2 = e;
+  if (splits == 1) e2.split_part = nullptr;
+  if (bn == 128) return launch_bn<128>(a, b, M, N, K, splits, e2, status, s);
+  return launch_bn<64>(a, b, M, N, K, splits, e2, status, s);
 }
 
 }  // namespace lsh

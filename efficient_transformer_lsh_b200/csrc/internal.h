@@ -117,7 +117,12 @@ struct GemmEpi {
   int64_t ldo, row0;
   int L, H;
   int M;
+  // optional scratch of kGemmMaxSplits * M * N floats: a plain float32
+  // product with few tiles is then split along K (the splits' sums are added
+  // in a fixed order, so the result stays deterministic)
+  float* split_part;
 };
+constexpr int kGemmMaxSplits = 4;
 // K a multiple of 64, N a multiple of 64; rows past M are neither read into
 // the output nor written.
 cudaError_t launch_gemm_tc(const GemmOpHost& a, const GemmOpHost& b, int M, int N, int K,

@@ -171,10 +171,14 @@ struct FfWs {
   __nv_bfloat16* h;    // [ff_chunk, d_ff] hidden block
   __nv_bfloat16* dh;   // [ff_chunk, d_ff] its gradient
   float* part;         // partial column sums of the bias gradients
+  float* split;        // K-split partial sums of the weight gradients
 };
 size_t ff_part_bytes(const lsh_ff_problem& f) {
   const size_t S = ((size_t)f.ff_chunk + kSumRows - 1) / kSumRows;
   return align_up(S * (size_t)std::max(f.d_ff, 64 * f.H) * 4, 256);
+}
+size_t ff_split_bytes(const lsh_ff_problem& f) {
+  return align_up((size_t)kGemmMaxSplits * 64 * f.H * f.d_ff * 4, 256);
 }
 FfWs ff_carve(const lsh_ff_problem& f, void* ws) {
   FfWs w;
@@ -182,6 +186,7 @@ FfWs ff_carve(const lsh_ff_problem& f, void* ws) {
   w.h = (__nv_bfloat16*)ws;
   w.dh = (__nv_bfloat16*)((char*)ws + hb);
   w.part = (float*)((char*)ws + 2 * hb);
+  w.split = (float*)((char*)ws + 2 * hb + ff_part_bytes(f));
   return w;
 }
 
@@ -221,7 +226,7 @@ cudaError_t ff_out(const lsh_ff_problem& f, const __nv_bfloat16* h, const void* 
 }  // namespace
 
 size_t ff_ws_bytes(const lsh_ff_problem& f) {
-  return 2 * align_up((size_t)f.ff_chunk * f.d_ff * 2, 256) + ff_part_bytes(f);
+  return 2 * align_up((size_t)f.ff_chunk * f.d_ff * 2, 256) + ff_part_bytes(f) + ff_split_bytes(f);
 }
 
 cudaError_t launch_ff_fwd(const lsh_ff_problem& f, const void* x, const void* W1, const float* b1,
@@ -276,6 +281,7 @@ cudaError_t launch_ff_bwd(const lsh_ff_problem& f, const void* x, const void* W1
       ep.accumulate = acc;
       ep.ldo = D;
       ep.M = f.d_ff;
+      ep.split_part = w.split;
       e = launch_gemm_tc(plain_op(w.h, Mc, f.d_ff, 1), heads_op(dy, f, 1, r0), f.d_ff, D, Mc, ep,
                          status, s);
       if (e != cudaSuccess) return e;
@@ -288,6 +294,7 @@ cudaError_t launch_ff_bwd(const lsh_ff_problem& f, const void* x, const void* W1
       ep.accumulate = acc;
       ep.ldo = f.d_ff;
       ep.M = D;
+      ep.split_part = w.split;
       e = launch_gemm_tc(heads_op(x, f, 1, r0), plain_op(w.dh, Mc, f.d_ff, 1), D, f.d_ff, Mc, ep,
                          status, s);
       if (e != cudaSuccess) return e;

@@ -305,7 +305,9 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
-// D[tmem] (+)= A * B, issued by one thread, with each shared-memory
+// D[tmem] (+)= A * B. Called by all 32 lanes of a converged warp (elect.sync
+// picks the one lane that issues; a call from a partial warp would wait
+// forever in elect.sync), with each shared-memory
 // descriptor given as its two 32-bit words: lo = (address >> 4) | (LBO >> 4)
 // << 16, hi = the SBO / version / swizzle word (smem_desc's upper half).
 // Issuers keep per-tile `lo` words and add constant offsets (bytes / 16;
@@ -337,7 +339,8 @@ __device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint3
 constexpr uint32_t kDescHi1024 = (1024u >> 4) | (1u << 14) | (2u << 29);
 __host__ __device__ constexpr uint32_t desc_lbo(uint32_t lbo_bytes) { return ((lbo_bytes >> 4) & 0x3FFFu) << 16; }
 
-// Arrives on `bar` once every previously issued MMA of this thread is done.
+// Arrives on `bar` once every previously issued MMA is done; like the MMA
+// helpers, called by a whole converged warp (one elected lane commits).
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   if (elect_one()) asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
