@@ -142,7 +142,11 @@ def test_feed_forward_chunking_is_bit_identical():
             assert torch.allclose(a, b, rtol=1e-4, atol=1e-3)
 
 
-@pytest.mark.parametrize("B,H,L,dff,chunk", [(1, 2, 256, 256, 128), (2, 3, 384, 384, 256)])
+@pytest.mark.parametrize("B,H,L,dff,chunk", [
+    (1, 2, 256, 256, 128),
+    (2, 3, 384, 384, 256),
+    (2, 2, 512, 256, 1024),    # 16 K blocks per weight-gradient product: split along K
+])
 def test_feed_forward_backward_matches_oracle(B, H, L, dff, chunk):
     import torch
     from efficient_transformer_lsh_b200 import _lib
