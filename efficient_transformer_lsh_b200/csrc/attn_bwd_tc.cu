@@ -205,17 +205,20 @@ constexpr uint32_t kLboK = desc_lbo(16), kLboN = desc_lbo(kTile);
 // S^T = X_K X_qb^T and dP^T = V_K dO_qb^T of step g (buffer g & 1); commits `full`.
 __device__ __forceinline__ void bwd_issue_s(uint32_t tmem, uint32_t sl, int g, int qb, int nc,
                                             uint64_t* full) {
-  if (qb < nc) {
-    const uint32_t d = tmem + kColBuf + (uint32_t)(g & 1) * 128;
-    const uint32_t xk = sl + kX / 16 + kLboK, vk = sl + kV / 16 + kLboK;
-    const uint32_t xq = sl + (kX + qb * kTile) / 16 + kLboK, gq = sl + (kDo + qb * kTile) / 16 + kLboK;
+  if (elect_one()) {
+    if (qb < nc) {
+      const uint32_t d = tmem + kColBuf + (uint32_t)(g & 1) * 128;
+      const uint32_t xk = sl + kX / 16 + kLboK, vk = sl + kV / 16 + kLboK;
+      const uint32_t xq = sl + (kX + qb * kTile) / 16 + kLboK, gq = sl + (kDo + qb * kTile) / 16 + kLboK;
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      mma_ss_w(d, xk + 2 * ks, xq + 2 * ks, kDescHi1024, kIdKK, ks > 0);
-      mma_ss_w(d + 64, vk + 2 * ks, gq + 2 * ks, kDescHi1024, kIdKK, ks > 0);
+      for (int ks = 0; ks < 4; ++ks) {
+        mma_ss_raw(d, xk + 2 * ks, xq + 2 * ks, kDescHi1024, kIdKK, ks > 0);
+        mma_ss_raw(d + 64, vk + 2 * ks, gq + 2 * ks, kDescHi1024, kIdKK, ks > 0);
+      }
     }
+    mma_commit_raw(full);
   }
-  mma_commit(full);
+  __syncwarp();
 }
 // dV += P^T dO_qb ; dK += dS^T X_qb, P^T and dS^T from step g's TMEM buffer.
 __device__ __forceinline__ void bwd_issue_g(uint32_t tmem, uint32_t acc, uint32_t sl, int g, int qb,
@@ -223,21 +226,27 @@ __device__ __forceinline__ void bwd_issue_g(uint32_t tmem, uint32_t acc, uint32_
   const uint32_t pt = tmem + kColBuf + (uint32_t)(g & 1) * 128;
   const uint32_t gq = sl + (kDo + qb * kTile) / 16 + kLboN, xq = sl + (kX + qb * kTile) / 16 + kLboN;
   // packed queries 0-31 sit at columns 0-15, queries 32-63 at columns 32-47
+  if (elect_one()) {
 #pragma unroll
-  for (int ks = 0; ks < 4; ++ks) {
-    const uint32_t ca = 8 * ks + 16 * (ks >> 1);
-    mma_ts_w(acc, pt + ca, gq + 128 * ks, kDescHi1024, kIdKN, acc_v || ks > 0);
-    mma_ts_w(acc + 64, pt + 64 + ca, xq + 128 * ks, kDescHi1024, kIdKN, acc_k || ks > 0);
+    for (int ks = 0; ks < 4; ++ks) {
+      const uint32_t ca = 8 * ks + 16 * (ks >> 1);
+      mma_ts_raw(acc, pt + ca, gq + 128 * ks, kDescHi1024, kIdKN, acc_v || ks > 0);
+      mma_ts_raw(acc + 64, pt + 64 + ca, xq + 128 * ks, kDescHi1024, kIdKN, acc_k || ks > 0);
+    }
   }
+  __syncwarp();
 }
 // Query-side product dS[128 queries of the dS^T blocks at ds] X_K over the
 // keys [16 KS0, 16 KS1), into the dK columns at d.
 template <int KS0, int KS1>
 __device__ __forceinline__ void bwd_issue_r(uint32_t d, uint32_t ds, uint32_t sl, bool acc) {
   const uint32_t xk = sl + kX / 16 + kLboN;
+  if (elect_one()) {
 #pragma unroll
-  for (int ks = KS0; ks < KS1; ++ks)
-    mma_ss_w(d, ds + 128 * ks, xk + 128 * ks, kDescHi1024, kIdNN, acc || ks > KS0);
+    for (int ks = KS0; ks < KS1; ++ks)
+      mma_ss_raw(d, ds + 128 * ks, xk + 128 * ks, kDescHi1024, kIdNN, acc || ks > KS0);
+  }
+  __syncwarp();
 }
 __device__ __forceinline__ bool bwd_wait_p(BwdBar* bar, int g, volatile int* abort, int* status) {
   return __all_sync(0xffffffffu, mbar_wait(&bar->p_full[g & 1], (uint32_t)(g >> 1) & 1u, abort, status));

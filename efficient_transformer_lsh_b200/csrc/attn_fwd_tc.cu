@@ -162,30 +162,29 @@ __device__ __forceinline__ bool fwd_issue_s(FwdBar* bar, uint32_t tmem, uint32_t
   const uint32_t d = tmem + (uint32_t)b * kSCols;
   const bool has_prev = jb.p > 0, has_odd = 2 * jb.p + 1 < n_chunks;
   const uint32_t q = sl + kLboK;
-  if (has_prev) {
-    const uint32_t prev_x = pb >= 0 ? pre0 + (uint32_t)(pb * kPreBytes) / 16
-                                    : slot0 + (uint32_t)(((nn + kSlots - 1) % kSlots) * kSlotBytes + kTile) / 16;
+  const uint32_t prev_x = pb >= 0 ? pre0 + (uint32_t)(pb * kPreBytes) / 16
+                                  : slot0 + (uint32_t)(((nn + kSlots - 1) % kSlots) * kSlotBytes + kTile) / 16;
+  const uint32_t id_main = has_odd ? kIdS128 : kIdS64;
+  if (elect_one()) {
+    if (has_prev) {
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_ss_raw(d, q + 2 * ks, prev_x + kLboK + 2 * ks, kDescHi1024, kIdS64, ks > 0);
+    }
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks)
-      mma_ss_w(d, q + 2 * ks, prev_x + kLboK + 2 * ks, kDescHi1024, kIdS64, ks > 0);
+      mma_ss_raw(d + 64, q + 2 * ks, q + 2 * ks, kDescHi1024, id_main, ks > 0);
+    mma_commit_raw(&bar->s_full[b]);
   }
-  if (has_odd) {
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks)
-      mma_ss_w(d + 64, q + 2 * ks, q + 2 * ks, kDescHi1024, kIdS128, ks > 0);
-  } else {
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks)
-      mma_ss_w(d + 64, q + 2 * ks, q + 2 * ks, kDescHi1024, kIdS64, ks > 0);
-  }
-  mma_commit(&bar->s_full[b]);
+  __syncwarp();
   return true;
 }
-// O (+)= P[:, 64 keys] V_block with P from TMEM.
+// O (+)= P[:, 64 keys] V_block with P from TMEM; issued by the calling
+// (elected) thread.
 __device__ __forceinline__ void fwd_issue_pv(uint32_t d, uint32_t pa, uint32_t v_lo, bool acc) {
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks)
-    mma_ts_w(d, pa + ks * 8, v_lo + 128 * ks, kDescHi1024, kIdO, acc || ks > 0);
+    mma_ts_raw(d, pa + ks * 8, v_lo + 128 * ks, kDescHi1024, kIdO, acc || ks > 0);
 }
 
 template <bool kCausal>
@@ -355,12 +354,15 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __half* __restric
         const uint32_t d = tmem + kOCol + (uint32_t)b * 64;
         const uint32_t pa = tmem + (uint32_t)b * kSCols;
         // key block 0 (previous chunk) when present, then blocks 1 and 2
-        if (has_prev) fwd_issue_pv(d, pa, prev_v + kLboV, false);
-        fwd_issue_pv(d, pa + 32, sl + 2 * kTile / 16 + kLboV, has_prev);
-        if (has_odd) fwd_issue_pv(d, pa + 64, sl + 3 * kTile / 16 + kLboV, true);
-        mma_commit(&bar->p_free[b]);                    // P(n) consumed, O(n) ready
-        if (n >= 1) mma_commit(&bar->slot_free[(n - 1) % kSlots]);
-        if (cur_pre >= 0) mma_commit(&bar->pre_free[cur_pre]);
+        if (elect_one()) {
+          if (has_prev) fwd_issue_pv(d, pa, prev_v + kLboV, false);
+          fwd_issue_pv(d, pa + 32, sl + 2 * kTile / 16 + kLboV, has_prev);
+          if (has_odd) fwd_issue_pv(d, pa + 64, sl + 3 * kTile / 16 + kLboV, true);
+          mma_commit_raw(&bar->p_free[b]);                // P(n) consumed, O(n) ready
+          if (n >= 1) mma_commit_raw(&bar->slot_free[(n - 1) % kSlots]);
+          if (cur_pre >= 0) mma_commit_raw(&bar->pre_free[cur_pre]);
+        }
+        __syncwarp();
         cur = nxt;
         cur_pre = nxt_pre;
         have_cur = have_nxt;

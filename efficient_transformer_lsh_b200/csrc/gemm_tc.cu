@@ -149,11 +149,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
       tc_fence_after();
       const uint32_t alo = (smem_u32(sa + s * kATile) >> 4) | a_lbo;
       const uint32_t blo = (smem_u32(sb + s * kBTile) >> 4) | b_lbo;
+      if (elect_one()) {
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        mma_ss_w(tmem, alo + a_step * ks, blo + b_step * ks, kDescHi1024, idesc,
-                 (kb > 0 || ks > 0) ? 1u : 0u);
-      mma_commit(&bar->empty[s]);
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ss_raw(tmem, alo + a_step * ks, blo + b_step * ks, kDescHi1024, idesc,
+                     (kb > 0 || ks > 0) ? 1u : 0u);
+        mma_commit_raw(&bar->empty[s]);
+      }
+      __syncwarp();
     }
     mma_commit(&bar->acc_full);
   } else {

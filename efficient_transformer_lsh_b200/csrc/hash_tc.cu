@@ -239,11 +239,14 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
               const uint32_t a = x_lo + (uint32_t)(s * kXBytes) / 16;
               const uint32_t bd =
                   r_lo + (uint32_t)(rs * kRBlockBytes + j * 4 * kRBoxBytes) / 16;
+              if (elect_one()) {
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_ss_w(d, a + 2 * kk, bd + 128 * kk, kDescHi1024, idesc, kk > 0);
-              mma_commit(&bar->acc_full[w]);
-              if (b == n_blk - 1 && j == nsub - 1) mma_commit(&bar->x_empty[s]);
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_ss_raw(d, a + 2 * kk, bd + 128 * kk, kDescHi1024, idesc, kk > 0);
+                mma_commit_raw(&bar->acc_full[w]);
+                if (b == n_blk - 1 && j == nsub - 1) mma_commit_raw(&bar->x_empty[s]);
+              }
+              __syncwarp();
             }
           if (stream_r && ok) {
             mma_commit(&bar->r_empty[rs]);
