@@ -270,8 +270,7 @@ struct StepRank {
   int src, rank, len;
   bool live, last;
 };
-__device__ __forceinline__ StepRank rank_step(uint32_t b, int lane) {
-  const uint32_t key = warp_sort32(b == 0xffffffffu ? 0xffffffffu : (b << 5) | (uint32_t)lane, lane);
+__device__ __forceinline__ StepRank rank_sorted(uint32_t key, int lane) {
   StepRank r;
   r.live = key != 0xffffffffu;
   r.bucket = key >> 5;
@@ -285,6 +284,12 @@ __device__ __forceinline__ StepRank rank_step(uint32_t b, int lane) {
   r.rank = lane - seg0;
   r.len = r.rank + 1;
   return r;
+}
+__device__ __forceinline__ uint32_t step_key(uint32_t b, int lane) {
+  return warp_sort32(b == 0xffffffffu ? 0xffffffffu : (b << 5) | (uint32_t)lane, lane);
+}
+__device__ __forceinline__ StepRank rank_step(uint32_t b, int lane) {
+  return rank_sorted(step_key(b, lane), lane);
 }
 
 __global__ void __launch_bounds__(1024)
@@ -370,6 +375,9 @@ sort_bscan_kernel(int32_t* __restrict__ totals, int n_buckets) {
   block_exclusive_scan(totals + (int64_t)blockIdx.x * n_buckets, n_buckets, red);
 }
 
+// kCache: pass 1 keeps each step's sorted keys in shared memory (4 bytes a
+// position, after the counters), so pass 2 only ranks them again.
+template <bool kCache>
 __global__ void __launch_bounds__(1024)
 sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restrict__ counts,
                     const int32_t* __restrict__ bases, int32_t* __restrict__ perm, int L,
@@ -380,6 +388,7 @@ sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restric
   int32_t* base = reinterpret_cast<int32_t*>(sm + (size_t)W * n_buckets * 2);     // [nb]
   int32_t* pre = base + n_buckets;                                                 // [nb]
   int* red = pre + n_buckets;                                                      // [64]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(red + 64);                          // [W][PW]
   const int q = blockIdx.x % Q;
   const int64_t seg = blockIdx.x / Q;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -416,7 +425,9 @@ sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restric
   // pass 1: this warp's count of every bucket
   for (int st = 0; st < PW; st += 32) {
     const uint32_t b = load_bucket(sbk, i0 + st + lane, L, n_buckets, nullptr);
-    const StepRank r = rank_step(b, lane);
+    const uint32_t key = step_key(b, lane);
+    if (kCache) keys[w * PW + st + lane] = key;
+    const StepRank r = rank_sorted(key, lane);
     if (r.live && r.last) mine[r.bucket] = (uint16_t)(mine[r.bucket] + r.len);
     __syncwarp();
   }
@@ -434,8 +445,13 @@ sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restric
   // pass 2: every position to base + warp run + earlier steps + rank
   int32_t* out = perm + seg * L;
   for (int st = 0; st < PW; st += 32) {
-    const uint32_t b = load_bucket(sbk, i0 + st + lane, L, n_buckets, nullptr);
-    const StepRank r = rank_step(b, lane);
+    StepRank r;
+    if (kCache) {
+      r = rank_sorted(keys[w * PW + st + lane], lane);
+    } else {
+      const uint32_t b = load_bucket(sbk, i0 + st + lane, L, n_buckets, nullptr);
+      r = rank_step(b, lane);
+    }
     if (r.live) out[base[r.bucket] + mine[r.bucket] + r.rank] = (int32_t)(i0 + st + r.src);
     __syncwarp();
     if (r.live && r.last) mine[r.bucket] = (uint16_t)(mine[r.bucket] + r.len);
@@ -488,8 +504,12 @@ cudaError_t launch_sort(const lsh_problem& p, const int32_t* bucket, int32_t* pe
     cudaError_t e = cudaFuncSetAttribute(sort_count_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_count_k);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)g.smem);
+    const size_t key_bytes = (size_t)g.W * g.PW * 4;
+    const bool cache = g.smem + key_bytes <= (size_t)kSortSmemBudget;
+    auto scatter = cache ? sort_scatter_kernel<true> : sort_scatter_kernel<false>;
+    const size_t sm_scatter = cache ? g.smem + key_bytes : g.smem;
+    e = cudaFuncSetAttribute(scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sm_scatter);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)(S * g.Q);
     sort_count_kernel<<<grid, 1024, sm_count_k, s>>>(bucket, ws.counts, p.L, p.n_buckets, g.P,
@@ -499,7 +519,7 @@ cudaError_t launch_sort(const lsh_problem& p, const int32_t* bucket, int32_t* pe
                                                                        p.n_buckets, g.Q, rows);
       sort_bscan_kernel<<<(unsigned)S, 1024, 0, s>>>(ws.base, p.n_buckets);
     }
-    sort_scatter_kernel<<<grid, g.W * 32, g.smem, s>>>(bucket, ws.counts,
+    scatter<<<grid, g.W * 32, sm_scatter, s>>>(bucket, ws.counts,
                                                        g.scanned ? ws.base : nullptr, perm, p.L,
                                                        p.n_buckets, g.PW, g.P, g.Q);
     note_launch(g.scanned ? 4 : 2);
