@@ -77,7 +77,7 @@ sum3_kernel(const __nv_bfloat16* __restrict__ a, const float* __restrict__ g1,
 // kSumRows rows starting at y kSumRows; warp w of it adds rows w, w + 8, ...
 // (16-byte loads, 8 columns a thread), then the 8 warps' sums are added in
 // warp order into part[y][c]. Pass 2: db[c] (+)= the parts in y order.
-constexpr int kSumRows = 256;
+constexpr int kSumRows = 256, kSumU = 8;
 
 __global__ void __launch_bounds__(256)
 colsum_part_kernel(const __nv_bfloat16* __restrict__ src, int heads, int64_t r0, int rows, int N,
@@ -90,21 +90,35 @@ colsum_part_kernel(const __nv_bfloat16* __restrict__ src, int heads, int64_t r0,
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
   if (c < N) {
-    for (int r = lo + w; r < hi; r += 8) {
-      const int64_t g = r0 + r;
-      int64_t off;
-      if (heads) {
-        const int64_t b = g / L, l = g - b * L;
-        off = ((b * H + c / 64) * L + l) * 64 + (c & 63);
-      } else {
-        off = g * ld + c;
-      }
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + off));
-      const uint32_t v[4] = {u.x, u.y, u.z, u.w};
+    // kSumU rows' loads in flight per thread before any of them is added;
+    // the adds still run in row order
+    for (int r = lo + w; r < hi; r += 8 * kSumU) {
+      uint4 u[kSumU];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[2 * i] += bf_lo(v[i]);
-        acc[2 * i + 1] += bf_hi(v[i]);
+      for (int j = 0; j < kSumU; ++j) {
+        const int rr = r + 8 * j;
+        if (rr < hi) {
+          const int64_t g = r0 + rr;
+          int64_t off;
+          if (heads) {
+            const int64_t b = g / L, l = g - b * L;
+            off = ((b * H + c / 64) * L + l) * 64 + (c & 63);
+          } else {
+            off = g * ld + c;
+          }
+          u[j] = __ldg(reinterpret_cast<const uint4*>(src + off));
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kSumU; ++j) {
+        if (r + 8 * j < hi) {
+          const uint32_t v[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[2 * i] += bf_lo(v[i]);
+            acc[2 * i + 1] += bf_hi(v[i]);
+          }
+        }
       }
     }
   }
