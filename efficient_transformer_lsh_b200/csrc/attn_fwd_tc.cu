@@ -34,7 +34,8 @@
 //                over S.
 //                After publishing P, the warpgroup writes its previous job's
 //                output: O from TMEM scaled by 1/l, as fp16, in original token
-//                order, + lse_r (so the stores stay off the path from S to P).
+//                order (32-byte stores, whole sectors), + lse_r (so the stores
+//                stay off the path from S to P).
 // fp16 for P and V keeps P's rounding error at 2^-11 (bf16 would add about
 // 3e-3 to O on the 64K workload).
 #include <cuda_fp16.h>
@@ -127,6 +128,13 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// One 32-byte store (the address is 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
 }
 
 // Thread t copies 16-byte pieces 4*(t&1)..+3 of row t>>1 of a chunk tile into
@@ -405,16 +413,16 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __half* __restric
           mbar_arrive(&bar->o_free[wg]);
         }
         if (pend_write) {
+          // whole 32-byte sectors: 16 columns per 256-bit store
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            dst[4 * h + c] = make_uint4(pack_f16x2(__uint_as_float(o[8 * c + 0]) * pend_inv_l,
-                                                   __uint_as_float(o[8 * c + 1]) * pend_inv_l),
-                                        pack_f16x2(__uint_as_float(o[8 * c + 2]) * pend_inv_l,
-                                                   __uint_as_float(o[8 * c + 3]) * pend_inv_l),
-                                        pack_f16x2(__uint_as_float(o[8 * c + 4]) * pend_inv_l,
-                                                   __uint_as_float(o[8 * c + 5]) * pend_inv_l),
-                                        pack_f16x2(__uint_as_float(o[8 * c + 6]) * pend_inv_l,
-                                                   __uint_as_float(o[8 * c + 7]) * pend_inv_l));
+          for (int c = 0; c < 2; ++c) {
+            uint32_t w[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              w[k] = pack_f16x2(__uint_as_float(o[16 * c + 2 * k]) * pend_inv_l,
+                                __uint_as_float(o[16 * c + 2 * k + 1]) * pend_inv_l);
+            st_global_v8(dst + 4 * h + 2 * c, w);
+          }
         }
       }
       if (pend_write) lsepart[pend_row] = pend_lse;
