@@ -15,6 +15,7 @@
 // Warp roles (persistent CTA, one per SM, walking units of kUnit pairs of one
 // (batch, head, round) segment):
 //   warps 0-3  : producers — cp.async gathers of x and v rows through perm
+//                (four whole 128-byte rows per instruction, eight lanes a row)
 //                straight into the 128-byte-swizzled K-major layout of a
 //                5-slot ring (a unit's first pair also needs chunk 2p0-1,
 //                which goes to one of 3 rotating side buffers). v arrives
@@ -137,16 +138,21 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
                : "memory");
 }
 
-// Thread t copies 16-byte pieces 4*(t&1)..+3 of row t>>1 of a chunk tile into
-// their 128-byte-swizzled places.
+// Warp w copies rows 16 w .. 16 w + 15 of a chunk tile into their
+// 128-byte-swizzled places, four whole rows per instruction (eight lanes per
+// row, one 16-byte piece each). Lane j (and j + 16) holds the position of
+// row 16 w + j; called by the whole warp.
 template <typename T16>
-__device__ __forceinline__ void issue_row(const T16* __restrict__ src_row, uint8_t* tile,
-                                          int row, int half) {
-  const uint32_t base = smem_u32(tile) + row * 128;
+__device__ __forceinline__ void issue_rows(const T16* __restrict__ src, uint8_t* tile, int pos,
+                                           int w, int lane) {
+  const uint32_t base = smem_u32(tile);
+  const int rsub = lane >> 3, ch = lane & 7;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int ch = half * 4 + i;
-    cp_async16(base + (((uint32_t)ch ^ (uint32_t)(row & 7)) << 4), src_row + ch * 8);
+  for (int g = 0; g < 4; ++g) {
+    const int r = 16 * w + 4 * g + rsub;
+    const int ps = __shfl_sync(0xffffffffu, pos, 4 * g + rsub);
+    cp_async16(base + r * 128 + (((uint32_t)ch ^ (uint32_t)(r & 7)) << 4),
+               src + (int64_t)ps * 64 + ch * 8);
   }
 }
 
@@ -241,7 +247,8 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __half* __restric
   if (wgi == 0) {
     // ------------------------------------------------ producers
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
-    const int t = threadIdx.x, row = t >> 1, half = t & 1;
+    // lane j and j + 16 of warp w hold the positions of row 16 w + j
+    const int row = 16 * warp + (lane & 15);
     JobIter it(blockIdx.x, n_units, gridDim.x, units_per_seg, n_pairs);
     Job cur, nxt;
     bool have_cur = it.next(cur);
@@ -298,17 +305,17 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __half* __restric
       const __half* vb = v + bh * L * 64;
       if (use_pre) {
         uint8_t* pb = pres + pb_idx * kPreBytes;
-        if (half == 0) bar->kpos_pre[pb_idx][row] = pos_p;
-        issue_row(xb + (int64_t)pos_p * 64, pb, row, half);
-        issue_row(vb + (int64_t)pos_p * 64, pb + kTile, row, half);
+        if (lane < 16) bar->kpos_pre[pb_idx][row] = pos_p;
+        issue_rows(xb, pb, pos_p, warp, lane);
+        issue_rows(vb, pb + kTile, pos_p, warp, lane);
       }
-      if (half == 0) bar->kpos[s][row] = pos_e;
-      issue_row(xb + (int64_t)pos_e * 64, sl, row, half);
-      issue_row(vb + (int64_t)pos_e * 64, sl + 2 * kTile, row, half);
+      if (lane < 16) bar->kpos[s][row] = pos_e;
+      issue_rows(xb, sl, pos_e, warp, lane);
+      issue_rows(vb, sl + 2 * kTile, pos_e, warp, lane);
       if (has_odd) {
-        if (half == 0) bar->kpos[s][64 + row] = pos_o;
-        issue_row(xb + (int64_t)pos_o * 64, sl + kTile, row, half);
-        issue_row(vb + (int64_t)pos_o * 64, sl + 3 * kTile, row, half);
+        if (lane < 16) bar->kpos[s][64 + row] = pos_o;
+        issue_rows(xb, sl + kTile, pos_o, warp, lane);
+        issue_rows(vb, sl + 3 * kTile, pos_o, warp, lane);
       }
       cp_async_commit();
       have_cur = it.next(nxt);
