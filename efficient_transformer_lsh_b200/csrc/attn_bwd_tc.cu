@@ -676,6 +676,13 @@ __device__ __forceinline__ void add8_f16(float (&acc)[8], const uint4 w) {
   }
 }
 
+// Eight floats to a 32-byte aligned address in one store.
+__device__ __forceinline__ void st_global_v8f(float* p, const float (&w)[8]) {
+  asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(w[0]),
+               "f"(w[1]), "f"(w[2]), "f"(w[3]), "f"(w[4]), "f"(w[5]), "f"(w[6]), "f"(w[7])
+               : "memory");
+}
+
 // dv, dqk of every token: the sum over rounds of its partial rows (row pos
 // of segment bh * n_rounds + r), plus the R1 row that emap names where the
 // token opens a unit; dv also takes dout for a token that attended only to
@@ -686,7 +693,7 @@ sum_rounds_kernel(const __half* __restrict__ part_dv, const __half* __restrict__
                   const __half* __restrict__ edge, const int32_t* __restrict__ emap,
                   const float* __restrict__ lse, const __nv_bfloat16* __restrict__ dout,
                   float* __restrict__ dqk, float* __restrict__ dv, int L, int n_rounds,
-                  int64_t n_edge_rows, int64_t N, int* status) {
+                  int64_t n_edge_rows, int64_t N, int wide, int* status) {
   const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
   const int c8 = (threadIdx.x & 7) * 8;
   if (t >= N) return;
@@ -734,12 +741,19 @@ sum_rounds_kernel(const __half* __restrict__ part_dv, const __half* __restrict__
 #pragma unroll
   for (int e = 0; e < 8; ++e) fin = fin && isfinite(a[e]) && isfinite(b[e]);
   if (!fin) record_status(status, (int)LSH_ERR_RANGE);
-  float4* pv = reinterpret_cast<float4*>(dv + t * 64 + c8);
-  float4* pq = reinterpret_cast<float4*>(dqk + t * 64 + c8);
-  pv[0] = make_float4(a[0], a[1], a[2], a[3]);
-  pv[1] = make_float4(a[4], a[5], a[6], a[7]);
-  pq[0] = make_float4(b[0], b[1], b[2], b[3]);
-  pq[1] = make_float4(b[4], b[5], b[6], b[7]);
+  if (wide) {
+    // 32-byte aligned outputs: one 256-bit store per row piece, so every
+    // store instruction writes whole sectors
+    st_global_v8f(dv + t * 64 + c8, a);
+    st_global_v8f(dqk + t * 64 + c8, b);
+  } else {
+    float4* pv = reinterpret_cast<float4*>(dv + t * 64 + c8);
+    float4* pq = reinterpret_cast<float4*>(dqk + t * 64 + c8);
+    pv[0] = make_float4(a[0], a[1], a[2], a[3]);
+    pv[1] = make_float4(a[4], a[5], a[6], a[7]);
+    pq[0] = make_float4(b[0], b[1], b[2], b[3]);
+    pq[1] = make_float4(b[4], b[5], b[6], b[7]);
+  }
 }
 
 bool tc_eligible(const lsh_problem& p) {
@@ -821,7 +835,7 @@ cudaError_t launch_attn_bwd_tc(const lsh_problem& p, const void* qk, const void*
       units_per_seg, status);
   sum_rounds_kernel<<<(unsigned)((N * 8 + 255) / 256), 256, 0, s>>>(
       w.part_dv, w.part_dqk, w.edge, w.emap, lse, (const __nv_bfloat16*)dout, dqk, dv, p.L,
-      p.n_rounds, n_units * kM, N, status);
+      p.n_rounds, n_units * kM, N, (((uintptr_t)dqk | (uintptr_t)dv) & 31) == 0 ? 1 : 0, status);
   note_launch(3);
   return cudaGetLastError();
 }
