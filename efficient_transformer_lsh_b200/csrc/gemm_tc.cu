@@ -85,6 +85,14 @@ __device__ __forceinline__ void load_box(void* dst, const CUtensorMap* map, int 
     tma_load_4d(dst, map, blk * 64, (int32_t)row, 0, 0, bar);
 }
 
+// Eight floats (v[o .. o + 7]) to a 32-byte aligned address in one store.
+__device__ __forceinline__ void st_v8(float* p, const float (&v)[16], int o) {
+  asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(v[o]),
+               "f"(v[o + 1]), "f"(v[o + 2]), "f"(v[o + 3]), "f"(v[o + 4]), "f"(v[o + 5]),
+               "f"(v[o + 6]), "f"(v[o + 7])
+               : "memory");
+}
+
 // Tile t of the product: M tile fastest, then N tile, then K split.
 struct TileCoord {
   int m0, n0, z;
@@ -102,7 +110,7 @@ template <int BN>
 __global__ void __launch_bounds__(kThreads, GemmCfg<BN>::kCtasPerSm)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                GemmOpDev a, GemmOpDev b, int K, GemmEpi e, int tiles_m, int tiles_n, int splits,
-               int* status) {
+               int wide, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sa = smem;
@@ -255,11 +263,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(acc[k]);
         if (e.split_part) {
           // one K split's raw sums; split_reduce_kernel adds the splits
-          float4* op = reinterpret_cast<float4*>(
-              e.split_part + ((int64_t)tc.z * e.M + row) * e.ldo + c);
+          float* sp = e.split_part + ((int64_t)tc.z * e.M + row) * e.ldo + c;
+          if (wide) {
+            st_v8(sp, v, 0);
+            st_v8(sp + 8, v, 8);
+          } else {
+            float4* op = reinterpret_cast<float4*>(sp);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            op[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            for (int k = 0; k < 4; ++k)
+              op[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          }
           continue;
         }
         if (e.bias) {
@@ -300,17 +313,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
         }
         if (e.out_f32) {
           float4* op = reinterpret_cast<float4*>((float*)e.out + off);
+          if (e.accumulate) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            float4 o = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-            if (e.accumulate) {
+            for (int k = 0; k < 4; ++k) {
               const float4 pp = op[k];
-              o.x += pp.x;
-              o.y += pp.y;
-              o.z += pp.z;
-              o.w += pp.w;
+              v[4 * k] += pp.x;
+              v[4 * k + 1] += pp.y;
+              v[4 * k + 2] += pp.z;
+              v[4 * k + 3] += pp.w;
             }
-            op[k] = o;
+          }
+          if (wide) {
+            st_v8((float*)e.out + off, v, 0);
+            st_v8((float*)e.out + off + 8, v, 8);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              op[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
           }
         } else {
           uint32_t pk[8];
@@ -319,9 +338,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant_
             __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
             pk[k] = *reinterpret_cast<uint32_t*>(&h2);
           }
-          uint4* op = reinterpret_cast<uint4*>((__nv_bfloat16*)e.out + off);
-          op[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          op[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          if (wide) {
+            asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
+                             (__nv_bfloat16*)e.out + off),
+                         "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]),
+                         "r"(pk[6]), "r"(pk[7])
+                         : "memory");
+          } else {
+            uint4* op = reinterpret_cast<uint4*>((__nv_bfloat16*)e.out + off);
+            op[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            op[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
         }
       }
     }
@@ -391,8 +418,13 @@ cudaError_t launch_bn(const GemmOpHost& a, const GemmOpHost& b, int M, int N, in
   const int tiles_m = (M + kBM - 1) / kBM, tiles_n = N / BN;
   const int n_tiles = tiles_m * tiles_n * splits;
   const int grid = std::min(n_tiles, GemmCfg<BN>::kCtasPerSm * sm_count());
+  // 256-bit stores when every 16-column piece of a row starts on 32 bytes:
+  // the base pointers 32-byte aligned and plain rows a multiple of 16
+  // elements apart (head-layout rows are 64 elements)
+  const bool wide = ((uintptr_t)e.out & 31) == 0 && ((uintptr_t)e.split_part & 31) == 0 &&
+                    (e.out_heads || e.ldo % 16 == 0);
   gemm_tc_kernel<BN><<<grid, kThreads, smem, s>>>(ma, mb, da, db, K, e, tiles_m, tiles_n, splits,
-                                                   status);
+                                                   wide ? 1 : 0, status);
   note_launch();
   if (e.split_part) {
     const int64_t n4 = (int64_t)M * N / 4;
