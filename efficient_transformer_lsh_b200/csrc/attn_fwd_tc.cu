@@ -125,6 +125,32 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Packed float32 pairs: (a0, a1) * (b, b) + (c, c) and (a0, a1) + (b0, b1).
+__device__ __forceinline__ float2 fma2(float a0, float a1, float b, float c) {
+  uint64_t a, bb, cc, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(bb) : "f"(b));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(cc) : "f"(c));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(bb), "l"(cc));
+  float2 y;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(y.x), "=f"(y.y) : "l"(r));
+  return y;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t x, y, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b.x), "f"(b.y));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(x), "l"(y));
+  float2 z;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(z.x), "=f"(z.y) : "l"(r));
+  return z;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -480,10 +506,13 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __half* __restric
           for (int e = 0; e < 4; ++e) {
             const int i = 4 * i4 + e;
             const bool valid = blk_ok && (kCausal ? (kk[e] < qpos) : (kk[e] != qpos));
-            const float x = valid ? __uint_as_float(sv[c2][i]) : -INFINITY;
-            sv[c2][i] = __float_as_uint(x);
-            mx4[e] = fmaxf(mx4[e], x);
+            sv[c2][i] = valid ? sv[c2][i] : __float_as_uint(-INFINITY);
           }
+          // two 3-input maxima per four scores
+          mx4[i4 & 3] = max3(mx4[i4 & 3], __uint_as_float(sv[c2][4 * i4]),
+                             __uint_as_float(sv[c2][4 * i4 + 1]));
+          mx4[(i4 + 2) & 3] = max3(mx4[(i4 + 2) & 3], __uint_as_float(sv[c2][4 * i4 + 2]),
+                                   __uint_as_float(sv[c2][4 * i4 + 3]));
         }
         (void)col;
         if (c2 == 0) tmem_ld_wait();
@@ -494,21 +523,22 @@ attn_fwd_tc_kernel(const __nv_bfloat16* __restrict__ qk, const __half* __restric
       // pass 2: P = exp2(scale * (s - max)) as fp16 pairs into TMEM over S;
       // P column block kb lives at TMEM columns [32 kb, 32 kb + 32). The masked
       // values are still in registers, so nothing is read back.
-      float l4[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c2 = 0; c2 < 2; ++c2) {
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float e0 = ex2(fmaf(__uint_as_float(sv[c2][2 * e]), scale_log2, neg));
-          const float e1 = ex2(fmaf(__uint_as_float(sv[c2][2 * e + 1]), scale_log2, neg));
-          l4[e & 3] += e0 + e1;
-          pk[e] = pack_f16x2(e0, e1);
+          const float2 t = fma2(__uint_as_float(sv[c2][2 * e]), __uint_as_float(sv[c2][2 * e + 1]),
+                                scale_log2, neg);
+          const float2 p2 = make_float2(ex2(t.x), ex2(t.y));
+          l2[e & 1] = add2(l2[e & 1], p2);
+          pk[e] = pack_f16x2(p2.x, p2.y);
         }
         tmem_st16(sbuf + (uint32_t)(kb0 * 32 + c2 * 32), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
         tmem_st16(sbuf + (uint32_t)(kb0 * 32 + c2 * 32 + 16), *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
       }
-      const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      const float l = (l2[0].x + l2[0].y) + (l2[1].x + l2[1].y);
       {
         uint32_t z[32];
 #pragma unroll
