@@ -11,9 +11,11 @@ namespace lsh {
 constexpr int kD = 64;  // head size supported by every kernel
 
 // Records an error code in the device status word unless one is already
-// there: the first error of a sequence of launches is the one reported.
+// there: the first error of a sequence of launches is the one reported. A
+// plain read first, so that when many threads meet an error only the first
+// few contend for the word.
 __device__ __forceinline__ void record_status(int* status, int code) {
-  if (status) atomicCAS(status, 0, code);
+  if (status && *(volatile int*)status == 0) atomicCAS(status, 0, code);
 }
 
 // Widen 4 consecutive elements to float.
