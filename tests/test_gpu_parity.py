@@ -175,3 +175,32 @@ def test_sort_paths_bit_exact(B, H, n_r, L, nb):
     assert _lib.lsh_device_status() == 0
     ref = np.argsort(bucket.reshape(-1, L), axis=1, kind="stable").reshape(bucket.shape)
     assert np.array_equal(perm.cpu().numpy(), ref)
+
+
+@pytest.mark.gpu
+def test_backward_outputs_only_16_byte_aligned_are_bit_identical():
+    """dqk and dv 16-byte aligned but not 32 (the ABI's rule is 16): the round
+    sum then writes each row piece with two 128-bit stores instead of one
+    256-bit store, and the gradients must not change by a bit."""
+    import torch
+    from efficient_transformer_lsh_b200 import _lib
+    from efficient_transformer_lsh_b200.attention import LSHAttention
+    w = WORKLOADS["enwik8-64k-bf16"].with_sizes(H=2, L=1472, backward=True)
+    inp = generate(w)
+    dev = torch.device("cuda")
+    t = {k: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(torch.bfloat16)
+         for k, a in inp.items()}
+    run = LSHAttention(w.B, w.H, w.L, w.n_buckets, w.n_rounds, w.chunk, w.causal, w.dtype, w.d,
+                       w.scale, dev)
+    run.forward(t["qk"], t["v"], t["R"])
+    dqk, dv = (g.clone() for g in run.backward(t["qk"], t["v"], t["dO"]))
+    n = dqk.numel()
+    # 16 bytes past the allocations' (256-byte aligned) starts
+    dqk16 = torch.full((n + 4,), float("nan"), dtype=torch.float32, device=dev)[4:]
+    dv16 = torch.full((n + 4,), float("nan"), dtype=torch.float32, device=dev)[4:]
+    assert dqk16.data_ptr() % 32 == 16 and dv16.data_ptr() % 32 == 16
+    _lib.lsh_attn_bwd(run.p, t["qk"], t["v"], run.perm, run.out, run.out_lo, run.lse, t["dO"],
+                      dqk16, dv16, run.ws_bwd, run.ws_bwd_bytes)
+    torch.cuda.synchronize()
+    assert _lib.lsh_device_status() == 0
+    assert torch.equal(dqk16.view_as(dqk), dqk) and torch.equal(dv16.view_as(dv), dv)

@@ -267,3 +267,44 @@ def test_reversible_block_matches_oracle(causal):
     # and the inverse recovers the original inputs up to the roundings of y
     assert np.abs(_np(outs["x2"]) - x2).max() < 4 * U * max(1.0, np.abs(gy2).max())
     assert np.abs(_np(outs["x1"]) - x1).max() < 4 * U * max(1.0, np.abs(gy1).max()) + 2e-2
+
+
+def test_feed_forward_outputs_only_16_byte_aligned_are_bit_identical():
+    """Outputs 16-byte aligned but not 32 (the ABI's rule is 16): the GEMM
+    epilogue then stores each 16-column piece with two 128-bit stores instead
+    of one 256-bit store; y, dx, the reconstruction and the weight gradients
+    must not change by a bit."""
+    import torch
+    from efficient_transformer_lsh_b200 import _lib
+    rng = np.random.default_rng(11)
+    B, H, L, dff, chunk = 2, 2, 512, 256, 1024     # the weight gradients split along K
+    x = _to(rng.standard_normal((B, H, L, 64)), torch.bfloat16)
+    res = _to(rng.standard_normal((B, H, L, 64)), torch.bfloat16)
+    dy = _to(rng.standard_normal((B, H, L, 64)), torch.bfloat16)
+    W = _weights(rng, 64 * H, dff)
+    f = _lib.make_ff_problem(B, H, L, dff, chunk)
+    y = _ff_run(f, x, W, res)
+    dx, rec, g = _ff_bwd_run(f, x, W, dy, dres=res, y_in=y)
+
+    def off16(shape, dtype):
+        n = int(np.prod(shape))
+        pad = 16 // torch.tensor([], dtype=dtype).element_size()
+        t = torch.full((n + pad,), float("nan"), dtype=dtype, device=_dev())[pad:]
+        assert t.data_ptr() % 32 == 16
+        return t.view(shape)
+
+    W1, b1, W2, b2 = W
+    Wd = (_to(W1, torch.bfloat16), _to(b1, torch.float32), _to(W2, torch.bfloat16),
+          _to(b2, torch.float32))
+    n = _lib.lsh_ff_workspace_size(f)
+    ws = torch.empty(n, dtype=torch.uint8, device=_dev())
+    y2 = off16(x.shape, torch.bfloat16)
+    _lib.lsh_ff_fwd(f, x, *Wd, res, y2, ws, n)
+    dx2, rec2 = off16(x.shape, torch.bfloat16), off16(x.shape, torch.bfloat16)
+    g2 = [off16(t.shape, torch.float32) for t in g]
+    _lib.lsh_ff_bwd(f, x, *Wd, dy, res, y, rec2, dx2, g2[0], g2[1], g2[2], g2[3], ws, n)
+    torch.cuda.synchronize()
+    assert _lib.lsh_device_status() == 0
+    assert torch.equal(y2, y) and torch.equal(dx2, dx) and torch.equal(rec2, rec)
+    for a, b in zip(g2, g):
+        assert torch.equal(a, b)
