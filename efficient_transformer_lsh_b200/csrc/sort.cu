@@ -223,9 +223,10 @@ WarpGeo warp_geo(const lsh_problem& p) {
   int64_t Q = ((int64_t)p.L + P - 1) / P;
   g.scanned = Q * nb > kDirectCounts || S * Q < 148;
   if (g.scanned) {
-    // smaller blocks, about two CTAs per SM over all segments; the scan
-    // kernels then give each CTA its bases
-    P = std::min<int64_t>(32768, std::max<int64_t>(32 * g.W, S * p.L / 296));
+    // smaller blocks, about one CTA per SM over all segments (each CTA's
+    // fixed work grows with W x n_buckets, so fewer, longer CTAs pay when
+    // n_buckets is large); the scan kernels then give each CTA its bases
+    P = std::min<int64_t>(32768, std::max<int64_t>(32 * g.W, S * p.L / 148));
   }
   g.PW = (int)((P + 32 * g.W - 1) / (32 * g.W)) * 32;
   g.P = g.W * g.PW;
