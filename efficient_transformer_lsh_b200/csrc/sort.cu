@@ -231,7 +231,9 @@ WarpGeo warp_geo(const lsh_problem& p) {
   g.PW = (int)((P + 32 * g.W - 1) / (32 * g.W)) * 32;
   g.P = g.W * g.PW;
   g.Q = (int)(((int64_t)p.L + g.P - 1) / g.P);
-  g.smem = (size_t)g.W * nb * 2 + (size_t)nb * 8 + 64 * 4;
+  // per-warp counters, bucket bases, block prefixes (not on the scanned
+  // path, whose bases already include them) and 64 words of scratch
+  g.smem = (size_t)g.W * nb * 2 + (size_t)nb * (g.scanned ? 4 : 8) + 64 * 4;
   return g;
 }
 
@@ -360,10 +362,17 @@ sort_qscan_kernel(int32_t* __restrict__ counts, int32_t* __restrict__ totals, in
   const int64_t seg = k / n_buckets, b = k - seg * n_buckets;
   int32_t* c = counts + seg * Q * (int64_t)n_buckets + b;
   int run = 0;
-  for (int q = 0; q < Q; ++q) {
-    const int v = c[(int64_t)q * n_buckets];
-    c[(int64_t)q * n_buckets] = run;
-    run += v;
+  // eight blocks' counts loaded before any is replaced, so their latencies
+  // overlap
+  for (int q0 = 0; q0 < Q; q0 += 8) {
+    int v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = q0 + u < Q ? c[(int64_t)(q0 + u) * n_buckets] : 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (q0 + u < Q) c[(int64_t)(q0 + u) * n_buckets] = run;
+      run += v[u];
+    }
   }
   totals[k] = run;
 }
@@ -387,8 +396,8 @@ sort_scatter_kernel(const int32_t* __restrict__ bucket, const int32_t* __restric
   const int W = blockDim.x >> 5;
   uint16_t* cnt = reinterpret_cast<uint16_t*>(sm);                                // [W][nb]
   int32_t* base = reinterpret_cast<int32_t*>(sm + (size_t)W * n_buckets * 2);     // [nb]
-  int32_t* pre = base + n_buckets;                                                 // [nb]
-  int* red = pre + n_buckets;                                                      // [64]
+  int32_t* pre = base + n_buckets;                                                 // [nb], unless scanned
+  int* red = pre + (bases ? 0 : n_buckets);                                        // [64]
   uint32_t* keys = reinterpret_cast<uint32_t*>(red + 64);                          // [W][PW]
   const int q = blockIdx.x % Q;
   const int64_t seg = blockIdx.x / Q;
