@@ -221,6 +221,12 @@ WarpGeo warp_geo(const lsh_problem& p) {
   // a few blocks per segment (at most ~16) of 8K..32K positions
   int64_t P = std::min<int64_t>(32768, std::max<int64_t>(8192, ((int64_t)p.L + 15) / 16));
   int64_t Q = ((int64_t)p.L + P - 1) / P;
+  if (S * Q > 2 * 148 && p.L <= 32768) {
+    // more CTAs than one wave of two per SM: one block per segment instead
+    // (no ragged second block)
+    P = p.L;
+    Q = 1;
+  }
   g.scanned = Q * nb > kDirectCounts || S * Q < 148;
   if (g.scanned) {
     // smaller blocks, about one CTA per SM over all segments (each CTA's
