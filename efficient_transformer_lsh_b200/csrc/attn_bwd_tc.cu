@@ -68,7 +68,7 @@ namespace {
 using namespace tc;
 
 constexpr int kM = 64;
-constexpr int kUnit = 16;
+constexpr int kUnit = 8;
 constexpr int kSlots = 2;
 constexpr int kTile = 64 * 128;        // 64 rows x 64 16-bit values
 // slot: x0 x1 x2 | v0 v1 | d0 d1 d2
